@@ -1,0 +1,7 @@
+"""B200-native fused attention-KL divergence (StreamKL forward and recompute backward).
+
+The compute path is libstreamkl.so (sm_100a kernels behind a C ABI, see
+include/streamkl.h); ``streamkl`` is its thin Python binding.
+"""
+from .binding import (StreamKLError, bwd, fwd, query_device_status, set_wait_limit_ms,  # noqa: F401
+                       streamkl, workspace_size)

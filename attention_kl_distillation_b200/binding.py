@@ -1,0 +1,182 @@
+"""Python binding of libstreamkl (the C ABI in include/streamkl.h).
+
+Argument marshalling only: tensors are checked for dtype, device, shape and
+layout, and their pointers, sizes and the current CUDA stream are passed to
+the library.  Every step of the computation runs in the library's sm_100a
+kernels; there is no fallback.  Importing this module fails if the library
+has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import re
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libstreamkl.so"
+HEADER = _PKG.parent / "include" / "streamkl.h"
+
+if not LIB_PATH.exists():
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m attention_kl_distillation_b200.build` "
+        "(the CUDA library is required; there is no fallback path)")
+
+_lib = ctypes.CDLL(str(LIB_PATH))
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT, EDEVICE = range(6)
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("NQ", ctypes.c_int),
+                ("NK", ctypes.c_int), ("d1", ctypes.c_int), ("d2", ctypes.c_int),
+                ("causal", ctypes.c_int), ("s1", ctypes.c_float), ("s2", ctypes.c_float)]
+
+
+_vp = ctypes.c_void_p
+_pp = ctypes.POINTER(Problem)
+_lib.streamkl_fwd.argtypes = [_pp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.streamkl_fwd.restype = ctypes.c_int
+_lib.streamkl_bwd_workspace_size.argtypes = [_pp]
+_lib.streamkl_bwd_workspace_size.restype = ctypes.c_size_t
+_lib.streamkl_bwd.argtypes = [_pp] + [_vp] * 12 + [ctypes.c_size_t, _vp]
+_lib.streamkl_bwd.restype = ctypes.c_int
+_lib.streamkl_status_string.argtypes = [ctypes.c_int]
+_lib.streamkl_status_string.restype = ctypes.c_char_p
+_lib.streamkl_query_device_status.argtypes = [_vp]
+_lib.streamkl_query_device_status.restype = ctypes.c_int
+_lib.streamkl_set_wait_limit_ms.argtypes = [ctypes.c_int]
+_lib.streamkl_set_wait_limit_ms.restype = ctypes.c_int
+_lib.streamkl_abi_version.restype = ctypes.c_int
+
+
+class StreamKLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/streamkl.h declares."""
+    text = HEADER.read_text()
+    return sorted(set(re.findall(r"\b(streamkl_[a-z_0-9]+)\s*\(", text)))
+
+
+def status_string(st: int) -> str:
+    return _lib.streamkl_status_string(int(st)).decode()
+
+
+def set_wait_limit_ms(ms: int) -> None:
+    st = _lib.streamkl_set_wait_limit_ms(int(ms))
+    if st != OK:
+        raise StreamKLError(st, "streamkl_set_wait_limit_ms")
+
+
+def query_device_status(stream: torch.cuda.Stream | None = None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return _lib.streamkl_query_device_status(_vp(s.cuda_stream))
+
+
+def problem(B, H, NQ, NK, d1, d2, causal=False, s1=None, s2=None) -> Problem:
+    return Problem(int(B), int(H), int(NQ), int(NK), int(d1), int(d2), int(bool(causal)),
+                   float(s1) if s1 is not None else 0.0, float(s2) if s2 is not None else 0.0)
+
+
+def _ptr(t):
+    return _vp(t.data_ptr()) if t is not None else _vp(0)
+
+
+def _check_qk(Q1, K1, Q2, K2):
+    for n, t in (("Q1", Q1), ("K1", K1), ("Q2", Q2), ("K2", K2)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous CUDA bf16 tensor [B, H, N, d]")
+    B, H, NQ, d1 = Q1.shape
+    NK = K1.shape[2]
+    d2 = Q2.shape[3]
+    if K1.shape != (B, H, NK, d1) or Q2.shape != (B, H, NQ, d2) or K2.shape != (B, H, NK, d2):
+        raise ValueError("inconsistent shapes of Q1, K1, Q2, K2")
+    if len({Q1.device, K1.device, Q2.device, K2.device}) != 1:
+        raise ValueError("inputs must be on one device")
+    return B, H, NQ, NK, d1, d2
+
+
+def _stream(device):
+    return _vp(torch.cuda.current_stream(device).cuda_stream)
+
+
+def fwd(Q1, K1, Q2, K2, causal=False, s1=None, s2=None, out=None):
+    """L, LSE1, LSE2 (fp32 [B, H, NQ]) via streamkl_fwd on the current stream."""
+    B, H, NQ, NK, d1, d2 = _check_qk(Q1, K1, Q2, K2)
+    prob = problem(B, H, NQ, NK, d1, d2, causal, s1, s2)
+    if out is None:
+        out = tuple(torch.empty((B, H, NQ), dtype=torch.float32, device=Q1.device)
+                    for _ in range(3))
+    L, A, Bv = out
+    with torch.cuda.device(Q1.device):
+        st = _lib.streamkl_fwd(ctypes.byref(prob), _ptr(Q1), _ptr(K1), _ptr(Q2), _ptr(K2),
+                               _ptr(L), _ptr(A), _ptr(Bv), _stream(Q1.device))
+    if st != OK:
+        raise StreamKLError(st, "streamkl_fwd")
+    return L, A, Bv
+
+
+def workspace_size(B, H, NQ, NK, d1, d2, causal=False) -> int:
+    prob = problem(B, H, NQ, NK, d1, d2, causal)
+    return int(_lib.streamkl_bwd_workspace_size(ctypes.byref(prob)))
+
+
+def bwd(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, causal=False, s1=None, s2=None,
+        need=(True, True, True, True), workspace=None):
+    """dQ1, dK1, dQ2, dK2 (bf16, None where not needed) via streamkl_bwd."""
+    B, H, NQ, NK, d1, d2 = _check_qk(Q1, K1, Q2, K2)
+    for n, t in (("dL", dL), ("L", L), ("LSE1", LSE1), ("LSE2", LSE2)):
+        if t.dtype != torch.float32 or t.shape != (B, H, NQ) or not t.is_contiguous() \
+                or t.device != Q1.device:
+            raise ValueError(f"{n} must be a contiguous fp32 tensor [B, H, NQ] on the inputs' device")
+    prob = problem(B, H, NQ, NK, d1, d2, causal, s1, s2)
+    outs = [torch.empty_like(t) if want else None
+            for t, want in zip((Q1, K1, Q2, K2), need)]
+    ws_bytes = int(_lib.streamkl_bwd_workspace_size(ctypes.byref(prob)))
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q1.device)
+    elif workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError("workspace too small")
+    with torch.cuda.device(Q1.device):
+        st = _lib.streamkl_bwd(ctypes.byref(prob), _ptr(dL), _ptr(Q1), _ptr(K1), _ptr(Q2),
+                               _ptr(K2), _ptr(L), _ptr(LSE1), _ptr(LSE2), *map(_ptr, outs),
+                               _ptr(workspace), ctypes.c_size_t(workspace.numel()
+                                                                * workspace.element_size()),
+                               _stream(Q1.device))
+    if st != OK:
+        raise StreamKLError(st, "streamkl_bwd")
+    return tuple(outs)
+
+
+class _StreamKLFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, Q1, K1, Q2, K2, causal, s1, s2):
+        L, LSE1, LSE2 = fwd(Q1, K1, Q2, K2, causal, s1, s2)
+        ctx.save_for_backward(Q1, K1, Q2, K2, L, LSE1, LSE2)
+        ctx.cfg = (causal, s1, s2)
+        return L
+
+    @staticmethod
+    def backward(ctx, dL):
+        Q1, K1, Q2, K2, L, LSE1, LSE2 = ctx.saved_tensors
+        causal, s1, s2 = ctx.cfg
+        need = tuple(bool(x) for x in ctx.needs_input_grad[:4])
+        if not any(need):
+            return (None,) * 7
+        grads = bwd(dL.float().contiguous(), Q1, K1, Q2, K2, L, LSE1, LSE2, causal, s1, s2,
+                    need=need)
+        return (*grads, None, None, None)
+
+
+def streamkl(Q1, K1, Q2, K2, causal=False, s1=None, s2=None):
+    """Row-wise KL(P1 || P2) [B, H, NQ] (fp32) with autograd support."""
+    return _StreamKLFunction.apply(Q1, K1, Q2, K2, causal, s1, s2)

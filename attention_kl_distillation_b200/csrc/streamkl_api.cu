@@ -1,0 +1,260 @@
+// streamkl_api.cu -- the C ABI of libstreamkl (declared in include/streamkl.h).
+//
+// Host-side only: argument validation, device capability checks, TMA
+// descriptor construction (cached per pointer and shape), and kernel launches
+// on the caller's stream.  No device memory is allocated here; the backward's
+// accumulator lives in a caller-provided workspace.
+#include "streamkl.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+
+namespace {
+
+__device__ int g_device_status;  // set by kernels (atomicCAS from 0), read + cleared by the host
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool sm100 = false;
+  int num_sms = 0;
+  int* status = nullptr;  // device address of g_device_status
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+unsigned long long g_wait_limit_ns = 0;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+unsigned long long wait_limit_ns() {
+  if (g_wait_limit_ns == 0) {
+    long ms = 2000;
+    if (const char* e = std::getenv("STREAMKL_WAIT_LIMIT_MS")) {
+      long v = std::strtol(e, nullptr, 10);
+      if (v >= 1) ms = v;
+    }
+    g_wait_limit_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+  }
+  return g_wait_limit_ns;
+}
+
+// Device of the current thread, probed once: sm_100 check, SM count, status word.
+streamkl_status current_device(DeviceInfo** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return STREAMKL_ECUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return STREAMKL_ECUDA;
+    d.sm100 = (prop.major == 10 && prop.minor == 0);
+    d.num_sms = prop.multiProcessorCount;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return STREAMKL_ECUDA;
+    d.status = static_cast<int*>(addr);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return STREAMKL_ECUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.probed = true;
+  }
+  if (!d.sm100) return STREAMKL_EUNSUPPORTED;
+  *out = &d;
+  return STREAMKL_OK;
+}
+
+// ------------------------------------------------------------ TMA descriptors
+struct MapKey {
+  const void* ptr;
+  int64_t BH, N;
+  int d, rows;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && BH == o.BH && N == o.N && d == o.d && rows == o.rows;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool used;
+};
+constexpr int kMapCache = 64;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+
+// 3-D map over a contiguous bf16 tensor [BH][N][d]: boxes of 64 elements of d
+// (128 bytes, the 128B-swizzle span) by `rows` rows by one head.
+streamkl_status tensor_map(const void* ptr, int64_t BH, int64_t N, int d, int rows,
+                           CUtensorMap* out) {
+  MapKey key{ptr, BH, N, d, rows};
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto& e : g_maps)
+    if (e.used && e.key == key) {
+      *out = e.map;
+      return STREAMKL_OK;
+    }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMap m;
+  CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return STREAMKL_ECUDA;
+  MapEntry& e = g_maps[g_map_next];
+  g_map_next = (g_map_next + 1) % kMapCache;
+  e.key = key;
+  e.map = m;
+  e.used = true;
+  *out = m;
+  return STREAMKL_OK;
+}
+
+// ------------------------------------------------------------ validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+streamkl_status check_problem(const streamkl_problem* pr) {
+  if (!pr) return STREAMKL_EINVAL;
+  if (pr->B < 1 || pr->H < 1 || pr->NQ < 1 || pr->NK < 1) return STREAMKL_EINVAL;
+  if (pr->causal != 0 && pr->causal != 1) return STREAMKL_EINVAL;
+  if (pr->causal && pr->NQ > pr->NK) return STREAMKL_EINVAL;
+  if (!std::isfinite(pr->s1) || !std::isfinite(pr->s2)) return STREAMKL_EINVAL;
+  // TMA coordinates are 32-bit signed; head count also indexes the grid.
+  const int64_t BH = static_cast<int64_t>(pr->B) * pr->H;
+  if (BH > (1 << 30) || pr->NQ > (1 << 30) || pr->NK > (1 << 30)) return STREAMKL_EINVAL;
+  if (BH * static_cast<int64_t>((pr->NQ + 127) / 128) > (1ll << 31) - 1) return STREAMKL_EINVAL;
+  if (!((pr->d1 == 64 || pr->d1 == 128) && (pr->d2 == 64 || pr->d2 == 128)))
+    return STREAMKL_EUNSUPPORTED;
+  return STREAMKL_OK;
+}
+
+float scale_or_default(float s, int d) {
+  return s > 0.f ? s : 1.0f / std::sqrt(static_cast<float>(d));
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+
+extern "C" {
+
+int streamkl_abi_version(void) { return 1; }
+
+const char* streamkl_status_string(streamkl_status st) {
+  switch (st) {
+    case STREAMKL_OK: return "ok";
+    case STREAMKL_EINVAL: return "invalid argument";
+    case STREAMKL_EUNSUPPORTED: return "unsupported configuration or device";
+    case STREAMKL_ECUDA: return "CUDA error";
+    case STREAMKL_ETIMEOUT: return "kernel pipeline wait timed out";
+    case STREAMKL_EDEVICE: return "device-side error";
+  }
+  return "unknown status";
+}
+
+streamkl_status streamkl_set_wait_limit_ms(int ms) {
+  if (ms < 1) return STREAMKL_EINVAL;
+  g_wait_limit_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+  return STREAMKL_OK;
+}
+
+streamkl_status streamkl_query_device_status(streamkl_stream_t stream) {
+  DeviceInfo* dev = nullptr;
+  streamkl_status st = current_device(&dev);
+  if (st != STREAMKL_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return STREAMKL_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof v) != cudaSuccess) return STREAMKL_ECUDA;
+  if (v != 0) {
+    int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero) != cudaSuccess)
+      return STREAMKL_ECUDA;
+  }
+  if (v == 0) return STREAMKL_OK;
+  if (v == STREAMKL_ETIMEOUT) return STREAMKL_ETIMEOUT;
+  return STREAMKL_EDEVICE;
+}
+
+streamkl_status streamkl_fwd(const streamkl_problem* prob, const void* Q1, const void* K1,
+                             const void* Q2, const void* K2, float* L, float* LSE1, float* LSE2,
+                             streamkl_stream_t stream) {
+  streamkl_status st = check_problem(prob);
+  if (st != STREAMKL_OK) return st;
+  const void* ins[4] = {Q1, K1, Q2, K2};
+  for (const void* p : ins)
+    if (!p || !aligned16(p)) return STREAMKL_EINVAL;
+  if (!L || !LSE1 || !LSE2) return STREAMKL_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(L) | reinterpret_cast<uintptr_t>(LSE1) |
+       reinterpret_cast<uintptr_t>(LSE2)) & 3u)
+    return STREAMKL_EINVAL;
+
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != STREAMKL_OK) return st;
+
+  const int64_t BH = static_cast<int64_t>(prob->B) * prob->H;
+  skl::FwdParams p;
+  if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, skl::kFwdBQ, &p.tmQ1)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kFwdBK, &p.tmK1)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, skl::kFwdBQ, &p.tmQ2)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(K2, BH, prob->NK, prob->d2, skl::kFwdBK, &p.tmK2)) != STREAMKL_OK) return st;
+  p.L = L;
+  p.LSE1 = LSE1;
+  p.LSE2 = LSE2;
+  p.BH = static_cast<int>(BH);
+  p.NQ = prob->NQ;
+  p.NK = prob->NK;
+  p.causal = prob->causal;
+  p.c1 = scale_or_default(prob->s1, prob->d1) * kLog2e;
+  p.c2 = scale_or_default(prob->s2, prob->d2) * kLog2e;
+  p.status = dev->status;
+  p.wait_limit_ns = wait_limit_ns();
+  const int units = skl::fwd_units(p.BH, p.NQ);
+  const int grid = units < dev->num_sms ? units : dev->num_sms;
+  if (skl::launch_fwd(p, prob->d1, prob->d2, grid, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return STREAMKL_ECUDA;
+  return STREAMKL_OK;
+}
+
+size_t streamkl_bwd_workspace_size(const streamkl_problem* prob) {
+  if (check_problem(prob) != STREAMKL_OK) return 0;
+  const size_t BH = static_cast<size_t>(prob->B) * prob->H;
+  const size_t n = BH * static_cast<size_t>(prob->NQ) * static_cast<size_t>(prob->d1 + prob->d2);
+  return ((n * sizeof(float) + 255) / 256) * 256;
+}
+
+streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, const void* Q1,
+                             const void* K1, const void* Q2, const void* K2, const float* L,
+                             const float* LSE1, const float* LSE2, void* dQ1, void* dK1, void* dQ2,
+                             void* dK2, void* workspace, size_t ws_bytes,
+                             streamkl_stream_t stream) {
+  (void)prob; (void)dL; (void)Q1; (void)K1; (void)Q2; (void)K2; (void)L; (void)LSE1;
+  (void)LSE2; (void)dQ1; (void)dK1; (void)dQ2; (void)dK2; (void)workspace; (void)ws_bytes;
+  (void)stream;
+  return STREAMKL_EUNSUPPORTED;
+}
+
+}  // extern "C"

@@ -1,0 +1,131 @@
+/*
+ * streamkl.h -- C ABI of libstreamkl: fused single-pass attention KL
+ * divergence on NVIDIA B200 (sm_100a).
+ *
+ * Operation (StreamKL summary page, "Metodologia", section 1 "Formulazione
+ * Online"): for batch b, head h and query row i,
+ *
+ *   x1[i,j] = s1 * <Q1[i], K1[j]>,  x2[i,j] = s2 * <Q2[i], K2[j]>
+ *   P_t[i,:] = softmax over the visible keys of x_t[i,:]
+ *   LSE_t[i] = log sum_j exp(x_t[i,j])
+ *   L[i]     = KL(P1[i,:] || P2[i,:]) = sum_j P1 * ((x1 - LSE1) - (x2 - LSE2))   (nats)
+ *
+ * computed in one pass over the keys without materialising the N_Q x N_K
+ * maps.  The backward (section 2, "Strategia di Ricalcolo") regenerates the
+ * probabilities tile by tile from the saved L, LSE1 and LSE2 and returns the
+ * gradients of sum_i dL[i] * L[i] for both gradient configurations of the
+ * page (teacher fixed: dQ2/dK2; student fixed: dQ1/dK1).
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors are device pointers, contiguous, row-major:
+ *      Q1 [B][H][NQ][d1], K1 [B][H][NK][d1], Q2 [B][H][NQ][d2], K2 [B][H][NK][d2]
+ *    in bf16 (IEEE binary32 with the low 16 bits dropped), 16-byte aligned.
+ *  - Row vectors L, LSE1, LSE2, dL are fp32 [B][H][NQ].
+ *  - Causal masking is bottom-right aligned: key j is visible from row i when
+ *    j <= i + NK - NQ (the usual j <= i when NQ == NK).  Causal with NQ > NK
+ *    is rejected, since some rows would see no key.
+ *  - The caller owns every buffer.  The library allocates no device memory on
+ *    any call below; host-side it keeps a small cache of TMA descriptors.
+ *  - Calls are asynchronous on the given stream (a cudaStream_t; NULL is the
+ *    legacy default stream).  Argument errors are returned synchronously and
+ *    launch nothing.  A kernel that detects a stalled pipeline records
+ *    STREAMKL_ETIMEOUT in a device status word and exits;
+ *    streamkl_query_device_status reads it.
+ */
+#ifndef STREAMKL_H_
+#define STREAMKL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so the header needs no CUDA include. */
+typedef struct CUstream_st *streamkl_stream_t;
+
+typedef enum {
+  STREAMKL_OK = 0,
+  STREAMKL_EINVAL = 1,       /* bad argument: null/unaligned pointer, bad size, bad workspace */
+  STREAMKL_EUNSUPPORTED = 2, /* valid but not built: head dims other than 64/128, no sm_100 device */
+  STREAMKL_ECUDA = 3,        /* a CUDA runtime/driver call or a launch failed */
+  STREAMKL_ETIMEOUT = 4,     /* a kernel gave up on a pipeline wait (device status word) */
+  STREAMKL_EDEVICE = 5       /* any other error recorded by a kernel */
+} streamkl_status;
+
+/*
+ * Problem description.  B, H, NQ, NK >= 1; d1, d2 in {64, 128}; causal 0/1.
+ * s1, s2: softmax scales of the two distributions; a value <= 0 selects
+ * 1/sqrt(d_t).  The two distributions may have different head dimensions
+ * (teacher d1, student d2) but share B, H, NQ and NK.
+ */
+typedef struct {
+  int B, H, NQ, NK, d1, d2, causal;
+  float s1, s2;
+} streamkl_problem;
+
+/*
+ * Forward: L, LSE1, LSE2 [B][H][NQ] fp32 from Q1, K1, Q2, K2 (bf16).
+ * Section 1 of the page: the five running scalars m1, m2, l1, l2 and acc per
+ * row, finished as L = acc/l1 + LSE2 - LSE1 with LSE_t = m_t + log l_t; key
+ * tiles past the causal frontier are skipped.  L, LSE1 and LSE2 are also
+ * the saved state of section 2 that streamkl_bwd consumes.
+ * Errors: EINVAL (null or unaligned pointer, sizes out of range, causal with
+ * NQ > NK), EUNSUPPORTED (d not in {64,128}, device is not sm_100), ECUDA.
+ */
+streamkl_status streamkl_fwd(const streamkl_problem *prob, const void *Q1, const void *K1,
+                             const void *Q2, const void *K2, float *L, float *LSE1, float *LSE2,
+                             streamkl_stream_t stream);
+
+/*
+ * Workspace bytes that streamkl_bwd needs for this problem: an fp32 dQ
+ * accumulator [B][H][NQ][d1+d2] (section 2, "Fusione del Kernel": dQ is
+ * accumulated with atomics across key tiles) plus padding.  0 on a bad
+ * problem.
+ */
+size_t streamkl_bwd_workspace_size(const streamkl_problem *prob);
+
+/*
+ * Backward: gradients of sum_i dL[i] * L[i] (section 2).  Inputs are the
+ * forward inputs plus the saved L, LSE1, LSE2 from streamkl_fwd and the
+ * upstream dL (fp32 [B][H][NQ]).  Outputs dQ1, dK1, dQ2, dK2 are bf16 with the
+ * shapes of their inputs; any of them may be NULL, which skips it: dQ1 = dK1
+ * = NULL is the page's configuration 1 (teacher P1 fixed), dQ2 = dK2 = NULL
+ * its configuration 2 (student P2 fixed).  workspace must hold
+ * streamkl_bwd_workspace_size bytes of device memory, 256-byte aligned; its
+ * contents on entry do not matter and on exit are unspecified.  Gradients are
+ * not bitwise reproducible (fp32 atomics).
+ * Errors: as streamkl_fwd, plus EINVAL for a short or unaligned workspace or
+ * all four outputs NULL.
+ */
+streamkl_status streamkl_bwd(const streamkl_problem *prob, const float *dL, const void *Q1,
+                             const void *K1, const void *Q2, const void *K2, const float *L,
+                             const float *LSE1, const float *LSE2, void *dQ1, void *dK1, void *dQ2,
+                             void *dK2, void *workspace, size_t ws_bytes, streamkl_stream_t stream);
+
+/* Static English text for a status code. */
+const char *streamkl_status_string(streamkl_status st);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that
+ * kernels set when a pipeline wait times out.  Returns STREAMKL_OK when no
+ * kernel has recorded an error since the last call, else the recorded code.
+ */
+streamkl_status streamkl_query_device_status(streamkl_stream_t stream);
+
+/*
+ * Upper bound, in milliseconds, on any single wait inside a kernel before it
+ * gives up with STREAMKL_ETIMEOUT (default 2000; also read once from the
+ * environment variable STREAMKL_WAIT_LIMIT_MS).  Values < 1 are rejected.
+ */
+streamkl_status streamkl_set_wait_limit_ms(int ms);
+
+/* Version of this ABI: 1. */
+int streamkl_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STREAMKL_H_ */
