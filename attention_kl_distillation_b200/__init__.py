@@ -3,5 +3,5 @@
 The compute path is libstreamkl.so (sm_100a kernels behind a C ABI, see
 include/streamkl.h); ``streamkl`` is its thin Python binding.
 """
-from .binding import (StreamKLError, bwd, fwd, query_device_status, set_wait_limit_ms,  # noqa: F401
-                       streamkl, workspace_size)
+from .binding import (StreamKLError, bwd, fwd, launch_count, query_device_status,  # noqa: F401
+                      set_wait_limit_ms, streamkl, workspace_size)

@@ -40,7 +40,7 @@ _lib.streamkl_fwd.argtypes = [_pp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.streamkl_fwd.restype = ctypes.c_int
 _lib.streamkl_bwd_workspace_size.argtypes = [_pp]
 _lib.streamkl_bwd_workspace_size.restype = ctypes.c_size_t
-_lib.streamkl_bwd.argtypes = [_pp] + [_vp] * 12 + [ctypes.c_size_t, _vp]
+_lib.streamkl_bwd.argtypes = [_pp] + [_vp] * 13 + [ctypes.c_size_t, _vp]
 _lib.streamkl_bwd.restype = ctypes.c_int
 _lib.streamkl_status_string.argtypes = [ctypes.c_int]
 _lib.streamkl_status_string.restype = ctypes.c_char_p
@@ -49,6 +49,7 @@ _lib.streamkl_query_device_status.restype = ctypes.c_int
 _lib.streamkl_set_wait_limit_ms.argtypes = [ctypes.c_int]
 _lib.streamkl_set_wait_limit_ms.restype = ctypes.c_int
 _lib.streamkl_abi_version.restype = ctypes.c_int
+_lib.streamkl_launch_count.restype = ctypes.c_uint64
 
 
 class StreamKLError(RuntimeError):
@@ -69,6 +70,11 @@ def header_functions() -> list[str]:
 
 def status_string(st: int) -> str:
     return _lib.streamkl_status_string(int(st)).decode()
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(_lib.streamkl_launch_count())
 
 
 def set_wait_limit_ms(ms: int) -> None:
@@ -131,16 +137,26 @@ def workspace_size(B, H, NQ, NK, d1, d2, causal=False) -> int:
 
 
 def bwd(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, causal=False, s1=None, s2=None,
-        need=(True, True, True, True), workspace=None):
-    """dQ1, dK1, dQ2, dK2 (bf16, None where not needed) via streamkl_bwd."""
+        need=(True, True, True, True), workspace=None, out=None):
+    """dQ1, dK1, dQ2, dK2 (bf16, None where not needed) via streamkl_bwd.
+
+    ``out`` may pass preallocated gradient tensors (None entries are skipped);
+    ``workspace`` a preallocated device buffer of at least ``workspace_size`` bytes."""
     B, H, NQ, NK, d1, d2 = _check_qk(Q1, K1, Q2, K2)
     for n, t in (("dL", dL), ("L", L), ("LSE1", LSE1), ("LSE2", LSE2)):
         if t.dtype != torch.float32 or t.shape != (B, H, NQ) or not t.is_contiguous() \
                 or t.device != Q1.device:
             raise ValueError(f"{n} must be a contiguous fp32 tensor [B, H, NQ] on the inputs' device")
     prob = problem(B, H, NQ, NK, d1, d2, causal, s1, s2)
-    outs = [torch.empty_like(t) if want else None
-            for t, want in zip((Q1, K1, Q2, K2), need)]
+    if out is not None:
+        outs = list(out)
+        for o, t in zip(outs, (Q1, K1, Q2, K2)):
+            if o is not None and (o.shape != t.shape or o.dtype != torch.bfloat16
+                                  or not o.is_contiguous() or o.device != t.device):
+                raise ValueError("gradient outputs must match their inputs (bf16, contiguous)")
+    else:
+        outs = [torch.empty_like(t) if want else None
+                for t, want in zip((Q1, K1, Q2, K2), need)]
     ws_bytes = int(_lib.streamkl_bwd_workspace_size(ctypes.byref(prob)))
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q1.device)

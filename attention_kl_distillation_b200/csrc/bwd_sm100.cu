@@ -1,0 +1,666 @@
+// bwd_sm100.cu -- recompute backward of the fused attention-KL for sm_100a.
+//
+// StreamKL summary page, "Metodologia" section 2: the probabilities are
+// regenerated tile by tile from the saved LSE vectors, P_t = exp(x_t - LSE_t),
+// and every (query tile, key tile) pair is visited once; dQ is accumulated
+// with atomics across key tiles.  With g = dL, c = L:
+//
+//   dS1 = g * P1 * ((x1 - LSE1) - (x2 - LSE2) - L)      (student fixed: dQ1, dK1)
+//   dS2 = g * (P2 - P1)                                 (teacher fixed: dQ2, dK2)
+//   dQ_t = s_t dS_t K_t,   dK_t = s_t dS_t^T Q_t
+//
+// B200 mapping (one CTA per SM, persistent, units handed out dynamically):
+//   work unit   (bh, 128-key tile); inner loop over 64-query steps that see it
+//   warp 0      TMA producer: K1/K2 tile per unit; Q1/Q2 tile + per-row record
+//               (LSE1, LSE2, L, s*dL) per step into a 2-stage ring; also
+//               fetches the next unit index and publishes it to the other roles
+//   warp 1      TMEM owner and UMMA issuer, per step:
+//                 S1^T = K1 Q1^T, S2^T = K2 Q2^T           (M=128 keys, N=64)
+//                 dK_t += dS_t^T Q_t                        (M=128 keys, N=d_t)
+//                 dQ_t^T = K_t^T dS_t^T                     (M=d_t, N=64 queries)
+//               S for step t+1 is issued before the contractions of step t so
+//               that the tensor pipe works while dS is being formed.
+//   warps 2..5  dS warpgroup: thread j owns key j (TMEM lane j): loads its S1^T,
+//               S2^T rows, regenerates P1, P2 with exp2 on the MUFU pipe,
+//               forms s1*dS1 and s2*dS2 in bf16 and writes them once to shared
+//               memory in the 128B-swizzled layout that serves both as the
+//               K-major A operand of dK and the MN-major B operand of dQ^T.
+//   warps 6..9  dQ warpgroup: reads dQ^T (thread = feature index) and adds it
+//               into the fp32 workspace with coalesced reductions; at the end
+//               of a unit converts the dK accumulators to bf16 and stores them.
+// TMEM (512 columns): S1^T [0,64) S2^T [64,128) dK1 [128,128+d1) dK2 [..,+d2)
+//                     dQ1^T [384,448) dQ2^T [448,512).
+#include "kernels.h"
+#include "sm100.cuh"
+
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+namespace skl {
+namespace {
+
+constexpr int BK = kBwdBK;  // keys per unit
+constexpr int BQ = kBwdBQ;  // queries per step
+constexpr int NTHREADS = 320;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint32_t kColS1 = 0, kColS2 = 64, kColDK1 = 128, kColDQ1 = 384, kColDQ2 = 448;
+
+template <int D1, int D2>
+struct BwdLayout {
+  static constexpr int k1_bytes = BK * D1 * 2;
+  static constexpr int k2_bytes = BK * D2 * 2;
+  static constexpr int q1_bytes = BQ * D1 * 2;
+  static constexpr int q2_bytes = BQ * D2 * 2;
+  static constexpr int rr_bytes = BQ * kRowRec * 4;
+  static constexpr int qstage_bytes = q1_bytes + q2_bytes + rr_bytes;
+  static constexpr int ds_bytes = BK * BQ * 2;  // one dS^T tile, bf16 [128 keys][64 queries]
+  static constexpr int QSTAGES = 2;
+  static constexpr int DSBUF = 2;
+  static constexpr int k1_off = 0;
+  static constexpr int k2_off = k1_off + k1_bytes;
+  static constexpr int q_off = k2_off + k2_bytes;
+  static constexpr int ds_off = q_off + QSTAGES * qstage_bytes;
+  static constexpr int bar_off = ds_off + DSBUF * 2 * ds_bytes;
+  // kfull kempty qfull[Q] qempty[Q] sfull sempty dsfull[D] dsempty[D] dqfull dqempty dkfull
+  // dkempty ufull[2] uempty[2] drain
+  static constexpr int nbar = 2 + 2 * QSTAGES + 2 + 2 * DSBUF + 4 + 4 + 1;
+  static constexpr int misc_off = bar_off + nbar * 8;
+  static constexpr int total = misc_off + 32;
+  static constexpr int alloc = total + 1024;
+  static_assert(alloc <= 232448, "shared memory budget exceeded");
+  static_assert(k1_bytes % 1024 == 0 && k2_bytes % 1024 == 0 && q1_bytes % 1024 == 0 &&
+                    q2_bytes % 1024 == 0 && rr_bytes % 1024 == 0,
+                "operand tiles must stay 1024-byte aligned");
+};
+
+struct UnitB {
+  int bh, k0, qt0, nsteps;
+};
+
+__device__ __forceinline__ UnitB decode_unit(const BwdParams& p, int u) {
+  const int nkt = (p.NK + BK - 1) / BK;
+  UnitB w;
+  w.bh = u / nkt;  // head-major: few heads active at once keeps Q and dQacc in L2
+  const int kt = u % nkt;  // within a head, the key tiles with the most query steps first
+  w.k0 = kt * BK;
+  const int nqt = p.NQpad / BQ;
+  int qt0 = 0;
+  if (p.causal) {
+    const int first = w.k0 - (p.NK - p.NQ);  // first query row that sees key k0
+    qt0 = first > 0 ? first / BQ : 0;
+  }
+  w.qt0 = qt0;
+  w.nsteps = nqt - qt0;
+  return w;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// dS for one key row j and the 64 queries of a step; writes the bf16 rows of
+// s1*dS1^T and s2*dS2^T (128 B each) into the swizzled tiles.
+template <bool MASK>
+__device__ __forceinline__ void form_ds(const uint32_t (&s1)[BQ], const uint32_t (&s2)[BQ],
+                                        const float* rr, float c1, float c2, int j, int key,
+                                        int q0, int NK, int causal, int off, uint32_t ds1_row,
+                                        uint32_t ds2_row) {
+#pragma unroll
+  for (int c = 0; c < BQ / 8; ++c) {
+    uint32_t w1[4], w2[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float d1v[2], d2v[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = c * 8 + h * 2 + e;
+        const float4 r = *reinterpret_cast<const float4*>(rr + i * kRowRec);
+        const float g2 = rr[i * kRowRec + 4];
+        const float u1 = fmaf(__uint_as_float(s1[i]), c1, -r.x);
+        const float u2 = fmaf(__uint_as_float(s2[i]), c2, -r.y);
+        const float P1 = ex2(u1), P2 = ex2(u2);
+        const float t = fmaf(u1 - u2, kLn2, -r.z);
+        float a = r.w * (P1 * t);
+        float b = g2 * (P2 - P1);
+        if (MASK) {
+          const bool vis = key < NK && (!causal || key <= q0 + i + off);
+          a = vis ? a : 0.f;
+          b = vis ? b : 0.f;
+        }
+        d1v[e] = a;
+        d2v[e] = b;
+      }
+      w1[h] = pack_bf16(d1v[0], d1v[1]);
+      w2[h] = pack_bf16(d2v[0], d2v[1]);
+    }
+    const uint32_t sw = static_cast<uint32_t>((c ^ (j & 7)) << 4);
+    st_shared_v4(ds1_row + sw, w1[0], w1[1], w1[2], w1[3]);
+    st_shared_v4(ds2_row + sw, w2[0], w2[1], w2[2], w2[3]);
+  }
+}
+
+template <int D1, int D2>
+__global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_constant__ BwdParams p) {
+  using Lay = BwdLayout<D1, D2>;
+  constexpr int QST = Lay::QSTAGES;
+  constexpr int DSB = Lay::DSBUF;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off);
+  uint64_t* kfull = bars + 0;
+  uint64_t* kempty = bars + 1;
+  uint64_t* qfull = bars + 2;
+  uint64_t* qempty = qfull + QST;
+  uint64_t* sfull = qempty + QST;
+  uint64_t* sempty = sfull + 1;
+  uint64_t* dsfull = sempty + 1;
+  uint64_t* dsempty = dsfull + DSB;
+  uint64_t* dqfull = dsempty + DSB;
+  uint64_t* dqempty = dqfull + 1;
+  uint64_t* dkfull = dqempty + 1;
+  uint64_t* dkempty = dkfull + 1;
+  uint64_t* ufull = dkempty + 1;
+  uint64_t* uempty = ufull + 2;
+  uint64_t* drain = uempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::misc_off + 4);
+  volatile int* unit_slot = reinterpret_cast<volatile int*>(smem + Lay::misc_off + 8);  // [2]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(kfull, 1);
+    mbar_init(kempty, 1);
+    for (int s = 0; s < QST; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qempty[s], 1);
+    }
+    mbar_init(sfull, 1);
+    mbar_init(sempty, 4);
+    for (int s = 0; s < DSB; ++s) {
+      mbar_init(&dsfull[s], 4);
+      mbar_init(&dsempty[s], 1);
+    }
+    mbar_init(dqfull, 1);
+    mbar_init(dqempty, 4);
+    mbar_init(dkfull, 1);
+    mbar_init(dkempty, 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ufull[s], 1);
+      mbar_init(&uempty[s], 9);  // MMA thread + 4 dS warps + 4 dQ warps
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmQ1);
+    tma_prefetch_desc(&p.tmK1);
+    tma_prefetch_desc(&p.tmQ2);
+    tma_prefetch_desc(&p.tmK2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int nkt = (p.NK + BK - 1) / BK;
+  const int total = p.BH * nkt;
+  int* counter = reinterpret_cast<int*>(const_cast<float*>(p.rowrec) +
+                                        static_cast<size_t>(p.BH) * p.NQpad * kRowRec);
+  uint8_t* k1_s = smem + Lay::k1_off;
+  uint8_t* k2_s = smem + Lay::k2_off;
+  auto q1_s = [&](int s) { return smem + Lay::q_off + s * Lay::qstage_bytes; };
+  auto q2_s = [&](int s) { return smem + Lay::q_off + s * Lay::qstage_bytes + Lay::q1_bytes; };
+  auto rr_s = [&](int s) {
+    return reinterpret_cast<float*>(smem + Lay::q_off + s * Lay::qstage_bytes + Lay::q1_bytes +
+                                    Lay::q2_bytes);
+  };
+  auto ds1_s = [&](int b) { return smem + Lay::ds_off + b * 2 * Lay::ds_bytes; };
+  auto ds2_s = [&](int b) { return smem + Lay::ds_off + b * 2 * Lay::ds_bytes + Lay::ds_bytes; };
+  const int off = p.NK - p.NQ;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int us = 0, qs = 0;
+      uint32_t uph = 0, kph = 0, qph = 0;
+      uint32_t armed_k = 0, armed_q[QST] = {};
+      int next = blockIdx.x;
+      bool ok = true;
+      for (;;) {
+        const int u = next < total ? next : -1;
+        if (!(ok = mbar_wait(&uempty[us], uph ^ 1, ctl))) break;
+        unit_slot[us] = u;
+        mbar_arrive(&ufull[us]);
+        if (++us == 2) {
+          us = 0;
+          uph ^= 1;
+        }
+        if (u < 0) break;
+        const UnitB w = decode_unit(p, u);
+        if (!(ok = mbar_wait(kempty, kph ^ 1, ctl))) break;
+        mbar_arrive_expect_tx(kfull, Lay::k1_bytes + Lay::k2_bytes);
+#pragma unroll
+        for (int b = 0; b < D1 / 64; ++b)
+          tma_load_3d(k1_s + b * (BK * 128), &p.tmK1, kfull, b * 64, w.k0, w.bh);
+#pragma unroll
+        for (int b = 0; b < D2 / 64; ++b)
+          tma_load_3d(k2_s + b * (BK * 128), &p.tmK2, kfull, b * 64, w.k0, w.bh);
+        armed_k = kph + 1;
+        kph ^= 1;
+        for (int t = 0; t < w.nsteps; ++t) {
+          const int q0 = (w.qt0 + t) * BQ;
+          if (!(ok = mbar_wait(&qempty[qs], qph ^ 1, ctl))) break;
+          mbar_arrive_expect_tx(&qfull[qs], Lay::qstage_bytes);
+#pragma unroll
+          for (int b = 0; b < D1 / 64; ++b)
+            tma_load_3d(q1_s(qs) + b * (BQ * 128), &p.tmQ1, &qfull[qs], b * 64, q0, w.bh);
+#pragma unroll
+          for (int b = 0; b < D2 / 64; ++b)
+            tma_load_3d(q2_s(qs) + b * (BQ * 128), &p.tmQ2, &qfull[qs], b * 64, q0, w.bh);
+          bulk_load(rr_s(qs), p.rowrec + (static_cast<size_t>(w.bh) * p.NQpad + q0) * kRowRec,
+                    Lay::rr_bytes, &qfull[qs]);
+          armed_q[qs] = qph + 1;
+          if (++qs == QST) {
+            qs = 0;
+            qph ^= 1;
+          }
+        }
+        if (!ok) break;
+        next = static_cast<int>(gridDim.x) + atomicAdd(counter, 1);
+      }
+      if (!ok) {
+        volatile int zero = 0;
+        WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
+        if (armed_k) mbar_wait(kfull, armed_k - 1, dctl);
+        for (int s = 0; s < QST; ++s)
+          if (armed_q[s]) mbar_wait(&qfull[s], armed_q[s] - 1, dctl);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(BK, BQ);                // S^T: M=128 keys, N=64
+      constexpr uint32_t idK1 = idesc_bf16(BK, D1, 0, 1);         // dK1: B = Q1 MN-major
+      constexpr uint32_t idK2 = idesc_bf16(BK, D2, 0, 1);
+      constexpr uint32_t idQ1 = idesc_bf16(D1, BQ, 1, 1);         // dQ1^T: A = K1 MN-major
+      constexpr uint32_t idQ2 = idesc_bf16(D2, BQ, 1, 1);
+      const uint32_t k1a = smem_u32(k1_s), k2a = smem_u32(k2_s);
+      int us = 0, qs_s = 0, qs_r = 0, db = 0;
+      uint32_t uph = 0, kph = 0, qph_s = 0, sph = 0, dqph = 0, dkph = 0;
+      uint32_t dsph[DSB] = {};
+      bool ok = true;
+      for (;;) {
+        if (!(ok = mbar_wait(&ufull[us], uph, ctl))) break;
+        const int u = unit_slot[us];
+        mbar_arrive(&uempty[us]);
+        if (++us == 2) {
+          us = 0;
+          uph ^= 1;
+        }
+        if (u < 0) break;
+        const UnitB w = decode_unit(p, u);
+        if (!(ok = mbar_wait(kfull, kph, ctl))) break;
+        kph ^= 1;
+        auto issue_s = [&]() -> bool {
+          if (!mbar_wait(&qfull[qs_s], qph_s, ctl)) return false;
+          if (!mbar_wait(sempty, sph ^ 1, ctl)) return false;
+          tc_fence_after();
+          const uint32_t qa1 = smem_u32(q1_s(qs_s)), qa2 = smem_u32(q2_s(qs_s));
+#pragma unroll
+          for (int kk = 0; kk < D1 / 16; ++kk) {
+            const uint32_t o = (kk & 3) * 32;
+            umma_bf16_ss(tmem_base + kColS1,
+                         sdesc_sw128(k1a + (kk >> 2) * (BK * 128) + o, 16, 1024),
+                         sdesc_sw128(qa1 + (kk >> 2) * (BQ * 128) + o, 16, 1024), idS, kk > 0);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D2 / 16; ++kk) {
+            const uint32_t o = (kk & 3) * 32;
+            umma_bf16_ss(tmem_base + kColS2,
+                         sdesc_sw128(k2a + (kk >> 2) * (BK * 128) + o, 16, 1024),
+                         sdesc_sw128(qa2 + (kk >> 2) * (BQ * 128) + o, 16, 1024), idS, kk > 0);
+          }
+          umma_commit(sfull);
+          sph ^= 1;
+          if (++qs_s == QST) {
+            qs_s = 0;
+            qph_s ^= 1;
+          }
+          return true;
+        };
+        if (!(ok = issue_s())) break;
+        for (int t = 0; t < w.nsteps && ok; ++t) {
+          if (t + 1 < w.nsteps && !(ok = issue_s())) break;
+          if (!(ok = mbar_wait(&dsfull[db], dsph[db], ctl))) break;
+          dsph[db] ^= 1;
+          if (t == 0) {
+            if (!(ok = mbar_wait(dkempty, dkph ^ 1, ctl))) break;
+            dkph ^= 1;
+          }
+          if (!(ok = mbar_wait(dqempty, dqph ^ 1, ctl))) break;
+          dqph ^= 1;
+          tc_fence_after();
+          const uint32_t qa1 = smem_u32(q1_s(qs_r)), qa2 = smem_u32(q2_s(qs_r));
+          const uint32_t d1a = smem_u32(ds1_s(db)), d2a = smem_u32(ds2_s(db));
+          // dK_t += (s_t dS_t)^T Q_t : A = dS^T (K-major, 128B rows of 64 queries),
+          // B = Q_t read MN-major (features contiguous; 64-feature chunks 8 KB apart).
+#pragma unroll
+          for (int kk = 0; kk < BQ / 16; ++kk) {
+            if (p.want_dk1)
+              umma_bf16_ss(tmem_base + kColDK1, sdesc_sw128(d1a + kk * 32, 16, 1024),
+                           sdesc_sw128(qa1 + kk * 2048, BQ * 128, 1024), idK1, (t > 0 || kk > 0));
+            if (p.want_dk2)
+              umma_bf16_ss(tmem_base + kColDK1 + D1, sdesc_sw128(d2a + kk * 32, 16, 1024),
+                           sdesc_sw128(qa2 + kk * 2048, BQ * 128, 1024), idK2, (t > 0 || kk > 0));
+          }
+          // dQ_t^T = K_t^T (s_t dS_t)^T : A = K tile read MN-major (64-feature chunks
+          // 16 KB apart), B = dS^T read MN-major (64 queries contiguous per key).
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            if (p.want_dq1)
+              umma_bf16_ss(tmem_base + kColDQ1, sdesc_sw128(k1a + kk * 2048, BK * 128, 1024),
+                           sdesc_sw128(d1a + kk * 2048, BQ * 128, 1024), idQ1, kk > 0);
+            if (p.want_dq2)
+              umma_bf16_ss(tmem_base + kColDQ2, sdesc_sw128(k2a + kk * 2048, BK * 128, 1024),
+                           sdesc_sw128(d2a + kk * 2048, BQ * 128, 1024), idQ2, kk > 0);
+          }
+          umma_commit(dqfull);
+          umma_commit(&dsempty[db]);
+          umma_commit(&qempty[qs_r]);
+          if (++db == DSB) db = 0;
+          if (++qs_r == QST) qs_r = 0;
+        }
+        if (!ok) break;
+        umma_commit(dkfull);
+        umma_commit(kempty);
+      }
+      umma_commit(drain);
+      volatile int zero = 0;
+      WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
+      mbar_wait(drain, 0, dctl);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ dS warpgroup
+    const int quarter = warp & 3;
+    const int j = quarter * 32 + lane;  // key row within the tile
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    int us = 0, qs = 0, db = 0;
+    uint32_t uph = 0, qph = 0, sph = 0;
+    uint32_t dsph[DSB] = {};
+    bool ok = true;
+    for (;;) {
+      if (!(ok = mbar_wait(&ufull[us], uph, ctl))) break;
+      const int u = unit_slot[us];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&uempty[us]);
+      if (++us == 2) {
+        us = 0;
+        uph ^= 1;
+      }
+      if (u < 0) break;
+      const UnitB w = decode_unit(p, u);
+      const int key = w.k0 + j;
+      for (int t = 0; t < w.nsteps; ++t) {
+        const int q0 = (w.qt0 + t) * BQ;
+        if (!(ok = mbar_wait(&qfull[qs], qph, ctl))) break;  // per-row records of this step
+        if (!(ok = mbar_wait(sfull, sph, ctl))) break;
+        sph ^= 1;
+        tc_fence_after();
+        uint32_t a[BQ], b[BQ];
+        tmem_ld_32x32b_x32(tl + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+        tmem_ld_32x32b_x32(tl + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+        tmem_ld_32x32b_x32(tl + kColS2, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
+        tmem_ld_32x32b_x32(tl + kColS2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
+        tmem_ld_wait();
+        reg_fence(a);
+        reg_fence(b);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sempty);
+        if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
+        dsph[db] ^= 1;
+        const uint32_t r1 = smem_u32(ds1_s(db)) + j * 128, r2 = smem_u32(ds2_s(db)) + j * 128;
+        const bool masked =
+            (p.causal && q0 + off < w.k0 + BK - 1) || (w.k0 + BK > p.NK);
+        if (masked)
+          form_ds<true>(a, b, rr_s(qs), p.c1, p.c2, j, key, q0, p.NK, p.causal, off, r1, r2);
+        else
+          form_ds<false>(a, b, rr_s(qs), p.c1, p.c2, j, key, q0, p.NK, p.causal, off, r1, r2);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dsfull[db]);
+        if (++db == DSB) db = 0;
+        if (++qs == QST) {
+          qs = 0;
+          qph ^= 1;
+        }
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------------------------ dQ / dK warpgroup
+    const int quarter = warp & 3;
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    // dQ_t^T rows are features: M = 128 puts feature f in lane f; M = 64 puts
+    // features 16q..16q+15 in lanes 32q..32q+15.
+    const int f1 = (D1 == 128) ? quarter * 32 + lane : (lane < 16 ? quarter * 16 + lane : -1);
+    const int f2 = (D2 == 128) ? quarter * 32 + lane : (lane < 16 ? quarter * 16 + lane : -1);
+    const int ldq = D1 + D2;
+    int us = 0;
+    uint32_t uph = 0, dqph = 0, dkph = 0;
+    bool ok = true;
+    for (;;) {
+      if (!(ok = mbar_wait(&ufull[us], uph, ctl))) break;
+      const int u = unit_slot[us];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&uempty[us]);
+      if (++us == 2) {
+        us = 0;
+        uph ^= 1;
+      }
+      if (u < 0) break;
+      const UnitB w = decode_unit(p, u);
+      for (int t = 0; t < w.nsteps; ++t) {
+        const int q0 = (w.qt0 + t) * BQ;
+        if (!(ok = mbar_wait(dqfull, dqph, ctl))) break;
+        dqph ^= 1;
+        tc_fence_after();
+        uint32_t a[BQ], b[BQ];
+        if (p.want_dq1) {
+          tmem_ld_32x32b_x32(tl + kColDQ1, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+          tmem_ld_32x32b_x32(tl + kColDQ1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+        }
+        if (p.want_dq2) {
+          tmem_ld_32x32b_x32(tl + kColDQ2, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
+          tmem_ld_32x32b_x32(tl + kColDQ2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
+        }
+        tmem_ld_wait();
+        reg_fence(a);
+        reg_fence(b);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dqempty);
+        const int nvalid = min(BQ, p.NQ - q0);
+        float* base = p.dQacc + (static_cast<size_t>(w.bh) * p.NQ + q0) * ldq;
+        if (p.want_dq1 && f1 >= 0) {
+#pragma unroll
+          for (int i = 0; i < BQ; ++i)
+            if (i < nvalid) atomicAdd(base + static_cast<size_t>(i) * ldq + f1, __uint_as_float(a[i]));
+        }
+        if (p.want_dq2 && f2 >= 0) {
+#pragma unroll
+          for (int i = 0; i < BQ; ++i)
+            if (i < nvalid)
+              atomicAdd(base + static_cast<size_t>(i) * ldq + D1 + f2, __uint_as_float(b[i]));
+        }
+      }
+      if (!ok) break;
+      // Unit epilogue: dK accumulators (thread = key row) to bf16.
+      if (!(ok = mbar_wait(dkfull, dkph, ctl))) break;
+      dkph ^= 1;
+      tc_fence_after();
+      const int key = w.k0 + quarter * 32 + lane;
+      const bool row_ok = key < p.NK;
+      if (p.want_dk1) {
+        __nv_bfloat16* dst = p.dK1 + (static_cast<size_t>(w.bh) * p.NK + key) * D1;
+#pragma unroll
+        for (int c = 0; c < D1; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tl + kColDK1 + c, v);
+          tmem_ld_wait();
+          reg_fence(v);
+          if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 o;
+              o.x = pack_bf16(__uint_as_float(v[e + 0]), __uint_as_float(v[e + 1]));
+              o.y = pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+              o.z = pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+              o.w = pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+              *reinterpret_cast<uint4*>(dst + c + e) = o;
+            }
+          }
+        }
+      }
+      if (p.want_dk2) {
+        __nv_bfloat16* dst = p.dK2 + (static_cast<size_t>(w.bh) * p.NK + key) * D2;
+#pragma unroll
+        for (int c = 0; c < D2; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tl + kColDK1 + D1 + c, v);
+          tmem_ld_wait();
+          reg_fence(v);
+          if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 o;
+              o.x = pack_bf16(__uint_as_float(v[e + 0]), __uint_as_float(v[e + 1]));
+              o.y = pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+              o.z = pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+              o.w = pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+              *reinterpret_cast<uint4*>(dst + c + e) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dkempty);
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// Per-row records (LSE1*log2e, LSE2*log2e, L, s1*dL, s2*dL, 0, 0, 0) padded to
+// whole 64-row steps with zeros (zero weight makes padded rows contribute
+// nothing), the zeroed dQ accumulator and the unit counter.
+__global__ void streamkl_bwd_prep_kernel(const BwdPrepParams p) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long nrec = static_cast<long long>(p.BH) * p.NQpad;
+  constexpr float kLog2e = 1.4426950408889634f;
+  for (long long r = tid; r < nrec; r += stride) {
+    const int bh = static_cast<int>(r / p.NQpad);
+    const int i = static_cast<int>(r % p.NQpad);
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < p.NQ) {
+      const size_t o = static_cast<size_t>(bh) * p.NQ + i;
+      const float g = p.dL[o];
+      a = make_float4(p.LSE1[o] * kLog2e, p.LSE2[o] * kLog2e, p.L[o], p.s1 * g);
+      b.x = p.s2 * g;
+    }
+    reinterpret_cast<float4*>(p.rowrec)[2 * r] = a;
+    reinterpret_cast<float4*>(p.rowrec)[2 * r + 1] = b;
+  }
+  const long long n4 = p.dqacc_elems / 4;
+  for (long long e = tid; e < n4; e += stride)
+    reinterpret_cast<float4*>(p.dQacc)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tid == 0) *reinterpret_cast<int*>(p.rowrec + nrec * kRowRec) = 0;
+}
+
+// fp32 dQ accumulator [rows][d1 + d2] -> bf16 dQ1 [rows][d1], dQ2 [rows][d2].
+__global__ void streamkl_bwd_convert_kernel(const BwdConvertParams p) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const int ld = p.d1 + p.d2;
+  const long long chunks = p.rows * (ld / 8);
+  for (long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks;
+       c += stride) {
+    const long long r = c / (ld / 8);
+    const int col = static_cast<int>(c % (ld / 8)) * 8;
+    const float4* src = reinterpret_cast<const float4*>(p.dQacc + r * ld + col);
+    const float4 x = src[0], y = src[1];
+    uint4 o;
+    o.x = pack_bf16(x.x, x.y);
+    o.y = pack_bf16(x.z, x.w);
+    o.z = pack_bf16(y.x, y.y);
+    o.w = pack_bf16(y.z, y.w);
+    if (col < p.d1) {
+      if (p.dQ1) *reinterpret_cast<uint4*>(p.dQ1 + r * p.d1 + col) = o;
+    } else {
+      if (p.dQ2) *reinterpret_cast<uint4*>(p.dQ2 + r * p.d2 + (col - p.d1)) = o;
+    }
+  }
+}
+
+template <int D1, int D2>
+cudaError_t launch_t(const BwdParams& p, int grid, cudaStream_t stream) {
+  constexpr int smem = BwdLayout<D1, D2>::alloc;
+  auto kern = streamkl_bwd_kernel<D1, D2>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, NTHREADS, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_smem_bytes(int d1, int d2) {
+  if (d1 == 128 && d2 == 128) return BwdLayout<128, 128>::alloc;
+  if (d1 == 128 && d2 == 64) return BwdLayout<128, 64>::alloc;
+  if (d1 == 64 && d2 == 128) return BwdLayout<64, 128>::alloc;
+  if (d1 == 64 && d2 == 64) return BwdLayout<64, 64>::alloc;
+  return 0;
+}
+
+cudaError_t launch_bwd(const BwdParams& p, int d1, int d2, int grid, cudaStream_t stream) {
+  if (d1 == 128 && d2 == 128) return launch_t<128, 128>(p, grid, stream);
+  if (d1 == 128 && d2 == 64) return launch_t<128, 64>(p, grid, stream);
+  if (d1 == 64 && d2 == 128) return launch_t<64, 128>(p, grid, stream);
+  if (d1 == 64 && d2 == 64) return launch_t<64, 64>(p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_prep(const BwdPrepParams& p, int num_sms, cudaStream_t stream) {
+  streamkl_bwd_prep_kernel<<<num_sms * 4, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_convert(const BwdConvertParams& p, int num_sms, cudaStream_t stream) {
+  streamkl_bwd_convert_kernel<<<num_sms * 4, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace skl

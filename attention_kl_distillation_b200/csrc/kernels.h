@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <cstdint>
 
 namespace skl {
@@ -29,6 +30,52 @@ size_t fwd_smem_bytes(int d1, int d2);
 
 // Launch the forward kernel; returns the launch error.
 cudaError_t launch_fwd(const FwdParams& p, int d1, int d2, int grid, cudaStream_t stream);
+
+// Keys per backward work unit (UMMA M of S^T and dK) and queries per step.
+constexpr int kBwdBK = 128;
+constexpr int kBwdBQ = 64;
+// Per-query-row record the backward reads: LSE1*log2e, LSE2*log2e, L, s1*dL, s2*dL, pad.
+constexpr int kRowRec = 8;
+
+struct BwdParams {
+  CUtensorMap tmQ1, tmK1, tmQ2, tmK2;  // Q maps: 64-row boxes; K maps: 128-row boxes
+  const float* rowrec;  // [BH][NQpad][kRowRec], NQpad = NQ rounded up to kBwdBQ
+  float* dQacc;         // [BH][NQ][d1 + d2] fp32, zeroed before the main kernel
+  __nv_bfloat16* dK1;   // [BH][NK][d1] or null
+  __nv_bfloat16* dK2;   // [BH][NK][d2] or null
+  int BH, NQ, NK, NQpad, causal;
+  int want_dq1, want_dk1, want_dq2, want_dk2;
+  float c1, c2;  // s_t * log2(e)
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+struct BwdPrepParams {
+  const float* L;
+  const float* LSE1;
+  const float* LSE2;
+  const float* dL;
+  float* rowrec;
+  float* dQacc;
+  long long dqacc_elems;
+  int BH, NQ, NQpad;
+  float s1, s2;
+};
+
+struct BwdConvertParams {
+  const float* dQacc;
+  __nv_bfloat16* dQ1;  // may be null
+  __nv_bfloat16* dQ2;  // may be null
+  long long rows;      // BH * NQ
+  int d1, d2;
+};
+
+size_t bwd_smem_bytes(int d1, int d2);
+cudaError_t launch_bwd(const BwdParams& p, int d1, int d2, int grid, cudaStream_t stream);
+cudaError_t launch_bwd_prep(const BwdPrepParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_convert(const BwdConvertParams& p, int num_sms, cudaStream_t stream);
+
+__host__ __device__ inline int bwd_units(int BH, int NK) { return BH * ((NK + kBwdBK - 1) / kBwdBK); }
 
 // Work units of the forward: (bh, 128-row query tile) pairs.
 __host__ __device__ inline int fwd_units(int BH, int NQ) { return BH * ((NQ + kFwdBQ - 1) / kFwdBQ); }

@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -22,6 +23,8 @@ namespace {
 __device__ int g_device_status;  // set by kernels (atomicCAS from 0), read + cleared by the host
 
 constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_launches{0};
 
 struct DeviceInfo {
   bool probed = false;
@@ -156,11 +159,34 @@ float scale_or_default(float s, int d) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Backward workspace: fp32 dQ accumulator [BH][NQ][d1+d2], then the per-row
+// records [BH][NQpad][8] fp32, then the work-unit counter; each part starts on
+// a 256-byte boundary.
+struct BwdWorkspace {
+  size_t dqacc_elems, rowrec_off, total;
+  int NQpad;
+};
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+BwdWorkspace bwd_workspace_layout(const streamkl_problem& pr) {
+  BwdWorkspace w;
+  const size_t BH = static_cast<size_t>(pr.B) * pr.H;
+  w.NQpad = (pr.NQ + skl::kBwdBQ - 1) / skl::kBwdBQ * skl::kBwdBQ;
+  w.dqacc_elems = BH * static_cast<size_t>(pr.NQ) * static_cast<size_t>(pr.d1 + pr.d2);
+  w.rowrec_off = round256(w.dqacc_elems * sizeof(float));
+  const size_t rec = BH * static_cast<size_t>(w.NQpad) * skl::kRowRec * sizeof(float);
+  w.total = w.rowrec_off + round256(rec + sizeof(int));
+  return w;
+}
+
 }  // namespace
 
 extern "C" {
 
 int streamkl_abi_version(void) { return 1; }
+
+uint64_t streamkl_launch_count(void) { return g_launches.load(); }
 
 const char* streamkl_status_string(streamkl_status st) {
   switch (st) {
@@ -236,14 +262,13 @@ streamkl_status streamkl_fwd(const streamkl_problem* prob, const void* Q1, const
   if (skl::launch_fwd(p, prob->d1, prob->d2, grid, reinterpret_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return STREAMKL_ECUDA;
+  g_launches.fetch_add(1);
   return STREAMKL_OK;
 }
 
 size_t streamkl_bwd_workspace_size(const streamkl_problem* prob) {
   if (check_problem(prob) != STREAMKL_OK) return 0;
-  const size_t BH = static_cast<size_t>(prob->B) * prob->H;
-  const size_t n = BH * static_cast<size_t>(prob->NQ) * static_cast<size_t>(prob->d1 + prob->d2);
-  return ((n * sizeof(float) + 255) / 256) * 256;
+  return bwd_workspace_layout(*prob).total;
 }
 
 streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, const void* Q1,
@@ -251,10 +276,92 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
                              const float* LSE1, const float* LSE2, void* dQ1, void* dK1, void* dQ2,
                              void* dK2, void* workspace, size_t ws_bytes,
                              streamkl_stream_t stream) {
-  (void)prob; (void)dL; (void)Q1; (void)K1; (void)Q2; (void)K2; (void)L; (void)LSE1;
-  (void)LSE2; (void)dQ1; (void)dK1; (void)dQ2; (void)dK2; (void)workspace; (void)ws_bytes;
-  (void)stream;
-  return STREAMKL_EUNSUPPORTED;
+  streamkl_status st = check_problem(prob);
+  if (st != STREAMKL_OK) return st;
+  const void* ins[4] = {Q1, K1, Q2, K2};
+  for (const void* p : ins)
+    if (!p || !aligned16(p)) return STREAMKL_EINVAL;
+  const float* vecs[4] = {dL, L, LSE1, LSE2};
+  for (const float* v : vecs)
+    if (!v || (reinterpret_cast<uintptr_t>(v) & 3u)) return STREAMKL_EINVAL;
+  void* outs[4] = {dQ1, dK1, dQ2, dK2};
+  bool any = false;
+  for (void* o : outs) {
+    if (o && !aligned16(o)) return STREAMKL_EINVAL;
+    any = any || o != nullptr;
+  }
+  if (!any) return STREAMKL_EINVAL;
+  const BwdWorkspace lay = bwd_workspace_layout(*prob);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < lay.total)
+    return STREAMKL_EINVAL;
+
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != STREAMKL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  const int64_t BH = static_cast<int64_t>(prob->B) * prob->H;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dqacc = reinterpret_cast<float*>(ws);
+  float* rowrec = reinterpret_cast<float*>(ws + lay.rowrec_off);
+  const float s1 = scale_or_default(prob->s1, prob->d1);
+  const float s2 = scale_or_default(prob->s2, prob->d2);
+  const bool want_dq = dQ1 || dQ2;
+
+  skl::BwdPrepParams pp;
+  pp.L = L;
+  pp.LSE1 = LSE1;
+  pp.LSE2 = LSE2;
+  pp.dL = dL;
+  pp.rowrec = rowrec;
+  pp.dQacc = dqacc;
+  pp.dqacc_elems = want_dq ? lay.dqacc_elems : 0;
+  pp.BH = static_cast<int>(BH);
+  pp.NQ = prob->NQ;
+  pp.NQpad = lay.NQpad;
+  pp.s1 = s1;
+  pp.s2 = s2;
+  if (skl::launch_bwd_prep(pp, dev->num_sms, s) != cudaSuccess) return STREAMKL_ECUDA;
+  g_launches.fetch_add(1);
+
+  skl::BwdParams p;
+  if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, skl::kBwdBQ, &p.tmQ1)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kBwdBK, &p.tmK1)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, skl::kBwdBQ, &p.tmQ2)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(K2, BH, prob->NK, prob->d2, skl::kBwdBK, &p.tmK2)) != STREAMKL_OK) return st;
+  p.rowrec = rowrec;
+  p.dQacc = dqacc;
+  p.dK1 = static_cast<__nv_bfloat16*>(dK1);
+  p.dK2 = static_cast<__nv_bfloat16*>(dK2);
+  p.BH = static_cast<int>(BH);
+  p.NQ = prob->NQ;
+  p.NK = prob->NK;
+  p.NQpad = lay.NQpad;
+  p.causal = prob->causal;
+  p.want_dq1 = dQ1 != nullptr;
+  p.want_dk1 = dK1 != nullptr;
+  p.want_dq2 = dQ2 != nullptr;
+  p.want_dk2 = dK2 != nullptr;
+  p.c1 = s1 * kLog2e;
+  p.c2 = s2 * kLog2e;
+  p.status = dev->status;
+  p.wait_limit_ns = wait_limit_ns();
+  const int units = skl::bwd_units(p.BH, p.NK);
+  const int grid = units < dev->num_sms ? units : dev->num_sms;
+  if (skl::launch_bwd(p, prob->d1, prob->d2, grid, s) != cudaSuccess) return STREAMKL_ECUDA;
+  g_launches.fetch_add(1);
+
+  if (want_dq) {
+    skl::BwdConvertParams cp;
+    cp.dQacc = dqacc;
+    cp.dQ1 = static_cast<__nv_bfloat16*>(dQ1);
+    cp.dQ2 = static_cast<__nv_bfloat16*>(dQ2);
+    cp.rows = BH * prob->NQ;
+    cp.d1 = prob->d1;
+    cp.d2 = prob->d2;
+    if (skl::launch_bwd_convert(cp, dev->num_sms, s) != cudaSuccess) return STREAMKL_ECUDA;
+    g_launches.fetch_add(1);
+  }
+  return STREAMKL_OK;
 }
 
 }  // extern "C"

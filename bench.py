@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention-KL forward + recompute backward on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+streamkl_fwd (L, LSE1, LSE2) then streamkl_bwd (dQ1, dK1, dQ2, dK2).  The
+default workload is the forward+backward configuration B1 H32 N=16384
+d1=d2=128 causal with dL = 1/(B*H*NQ).  Inputs (537 MB) are larger than the
+126 MB L2, so no flush is needed between steps.
+
+Prints one JSON line (rank 0).  With torchrun (N > 1) every rank runs an
+independent replica of the workload (weak scaling: the path has no data
+exchange); the timed region is bracketed by barriers and the max over ranks
+is taken.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores on a
+bounded sample of the same workload (the only other place this file runs the
+oracle is the ``cpu_baseline`` leg).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import numpy as np
+import torch
+
+ROOT = Path(__file__).resolve().parent
+if str(ROOT) not in sys.path:
+    sys.path.insert(0, str(ROOT))
+
+from attention_kl_distillation_b200.inputs import WORKLOADS, Workload, bf16_bits, make_inputs  # noqa: E402
+
+METRIC = "fused attn-KL fwd / fwd+bwd TFLOP/s and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_TFLOPS = 1590.0
+FALLBACK_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fwdbwd16k")
+    ap.add_argument("--phase", choices=["auto", "fwd", "fwdbwd"], default="auto")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# --------------------------------------------------------------------------- helpers
+def peaks():
+    f = ROOT / "MEASURED_PEAKS.json"
+    try:
+        d = json.loads(f.read_text())
+        return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_TFLOPS, FALLBACK_GBS, "fallback"
+
+
+def host_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def workload_desc(w: Workload, phase: str) -> dict:
+    return {
+        "workload": (f"{w.name}: B{w.B} H{w.H} NQ={w.NQ} NK={w.NK} d1={w.d1} d2={w.d2} "
+                     f"{'causal' if w.causal else 'non-causal'}, "
+                     f"{'forward+backward' if phase == 'fwdbwd' else 'forward'}"),
+        "B": w.B, "H": w.H, "NQ": w.NQ, "NK": w.NK, "d1": w.d1, "d2": w.d2,
+        "causal": w.causal, "phase": phase,
+        "student": w.student + (f" sigma={w.sigma}" if w.student == "perturb" else ""),
+        "l2": f"inputs {w.input_bytes() / 1e6:.0f} MB vs 126 MB L2; "
+              + ("no flush (inputs larger than L2)" if w.input_bytes() > 126e6
+                 else "L2 flushed between steps"),
+    }
+
+
+def step_flops(w: Workload, phase: str) -> int:
+    return w.fwd_flops() + (w.bwd_flops() if phase == "fwdbwd" else 0)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.t0 = self.t1 = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def finish(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
+            except Exception:
+                continue
+        inside = [r for r in rows if self.t0 - 0.05 <= r[0] <= self.t1 + 0.05] or rows[-3:]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in inside for n, v in zip(names, r[3]) if v.lower() == "active"})
+        return {
+            "sm_mhz": statistics.median(r[1] for r in inside) if inside else None,
+            "sm_max_mhz": max(r[2] for r in inside) if inside else None,
+            "reasons": reasons,
+            "samples": len(inside),
+        }
+
+
+# --------------------------------------------------------------------------- oracle legs
+def oracle_sample_run(w: Workload, phase: str, R: int, nthreads: int, seed: int):
+    """Run the oracle on a bounded sample of the workload: the first R query rows of head 0
+    with the keys they can see (for a causal square problem that prefix is itself the problem
+    NQ = NK = R; otherwise R rows against all keys).  Returns (seconds, algorithmic FLOPs)."""
+    from oracle import oracle as O
+    orc = O.default()
+    sub = w.with_(B=1, H=1, NQ=R, NK=R if (w.causal and w.NQ == w.NK) else w.NK)
+    Q1, K1, Q2, K2 = (bf16_bits(t) for t in make_inputs(sub, seed=seed))
+    t0 = time.perf_counter()
+    if phase == "fwdbwd":
+        orc.fwd_all(Q1, K1, Q2, K2, causal=sub.causal, nthreads=nthreads)
+        g = np.full((1, sub.NQ), 1.0 / (w.B * w.H * w.NQ))
+        orc.bwd_heads(Q1, K1, Q2, K2, [0], g, causal=sub.causal, nthreads=nthreads)
+    else:
+        orc.fwd_all(Q1, K1, Q2, K2, causal=sub.causal, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return dt, step_flops(sub, phase), sub
+
+
+def cpu_baseline(w: Workload, phase: str, target_s: float) -> dict:
+    nthreads = host_threads()
+    R = 512
+    dt, fl, sub = oracle_sample_run(w, phase, R, nthreads, w.seed)
+    if dt < target_s / 4:
+        scale = (target_s / max(dt, 1e-3)) ** (0.5 if sub.NK == sub.NQ else 1.0)
+        R = int(min(w.NQ, max(R, R * scale * 0.9)) // 64 * 64)
+        dt, fl, sub = oracle_sample_run(w, phase, R, nthreads, w.seed)
+    return {
+        "value": fl / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+        "seconds": dt,
+        "sample": (f"first {sub.NQ} query rows of one head ({sub.NK} keys, "
+                   f"{'causal' if sub.causal else 'non-causal'}) of the {w.name} recipe, "
+                   f"{'forward+backward' if phase == 'fwdbwd' else 'forward'}; "
+                   f"{fl / 1e9:.1f} GFLOP algorithmic"),
+    }
+
+
+def run_reference(args, w: Workload, phase: str):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    nthreads = host_threads()
+    budget = 150.0 / max(1, args.steps + args.warmup)  # seconds of oracle work per step
+    R = 512
+    dt, fl, sub = oracle_sample_run(w, phase, R, nthreads, w.seed)
+    if dt < budget / 2:
+        scale = (budget / max(dt, 1e-3)) ** (0.5 if sub.NK == sub.NQ else 1.0)
+        R = int(min(w.NQ, max(R, R * scale * 0.8)) // 64 * 64)
+    times = []
+    for s in range(args.warmup + args.steps):
+        dt, fl, sub = oracle_sample_run(w, phase, R, nthreads, w.seed + s)
+        if s >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = fl * len(times) / total / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference", "config": workload_desc(w, phase),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": f"first {sub.NQ} query rows of one head per step "
+                                   f"({sub.NK} keys), {fl / 1e9:.1f} GFLOP algorithmic"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our path
+def main(argv=None):
+    args = parse_args(argv)
+    w = WORKLOADS[args.workload]
+    phase = args.phase if args.phase != "auto" else ("fwdbwd" if w.backward else "fwd")
+    if args.impl == "reference":
+        return run_reference(args, w, phase)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import attention_kl_distillation_b200 as skl
+    from attention_kl_distillation_b200 import binding
+
+    dev = torch.device("cuda", local)
+    cpu_ins = make_inputs(w, seed=w.seed + rank)  # independent replica per rank
+    Q1, K1, Q2, K2 = (t.to(dev) for t in cpu_ins)
+    g = 1.0 / (w.B * w.H * w.NQ)
+    dL = torch.full((w.B, w.H, w.NQ), g, device=dev)
+    L, A, B = (torch.empty((w.B, w.H, w.NQ), device=dev) for _ in range(3))
+    grads = tuple(torch.empty_like(t) for t in (Q1, K1, Q2, K2))
+    ws = torch.empty(binding.workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B))
+        if phase == "fwdbwd":
+            skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal, workspace=ws, out=grads)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if skl.query_device_status() != 0:
+        raise RuntimeError("device status reported an error after warm-up")
+
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = skl.launch_count()
+    clocks.mark_start()
+    t_start.record(stream)
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B))
+        ev[k][1].record(stream)
+        if phase == "fwdbwd":
+            skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal, workspace=ws, out=grads)
+        ev[k][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    barrier()
+    launches = skl.launch_count() - launches0
+    clk = clocks.finish()
+    if skl.query_device_status() != 0:
+        raise RuntimeError("device status reported an error in the timed region")
+
+    total_ms = t_start.elapsed_time(t_end)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) if phase == "fwdbwd" else 0.0
+    fl_step = step_flops(w, phase)
+    value = world * fl_step * args.steps / (total_ms * 1e-3) / 1e12
+    peak, hbm, src = peaks()
+    fwd_tf = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if bwd_ms > 0 else None
+    if phase == "fwdbwd" and bwd_ms >= fwd_ms:
+        dom = {"kernel": "streamkl_bwd (prep + main + dQ convert kernels)", "achieved": bwd_tf,
+               "flops_per_launch": w.bwd_flops(), "ms": bwd_ms}
+    else:
+        dom = {"kernel": "streamkl_fwd_kernel", "achieved": fwd_tf,
+               "flops_per_launch": w.fwd_flops(), "ms": fwd_ms}
+    roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": peak, "unit": UNIT,
+                "frac": dom["achieved"] / peak, "traffic": None, "kernel": dom["kernel"],
+                "flops_per_launch": dom["flops_per_launch"], "ms_per_launch": dom["ms"],
+                "peak_source": f"{src} dense bf16 (burst)"}
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        h_in = [t.pin_memory() for t in cpu_ins]
+        h_dL = dL.cpu().pin_memory()
+        h_L = torch.empty((w.B, w.H, w.NQ), dtype=torch.float32).pin_memory()
+        h_g = [torch.empty(t.shape, dtype=torch.bfloat16).pin_memory() for t in cpu_ins]
+        h2d = sum(t.numel() * t.element_size() for t in h_in) + h_dL.numel() * 4
+        d2h = h_L.numel() * 4 + (sum(t.numel() * 2 for t in h_g) if phase == "fwdbwd" else 0)
+
+        def e2e_step():
+            d_in = [t.to(dev, non_blocking=True) for t in h_in]
+            d_dL = h_dL.to(dev, non_blocking=True)
+            if phase == "fwdbwd":
+                Lx = skl.streamkl(*[t.requires_grad_(True) for t in d_in], causal=w.causal)
+                Lx.backward(d_dL)
+                for hg, t in zip(h_g, d_in):
+                    hg.copy_(t.grad, non_blocking=True)
+            else:
+                Lx, _, _ = skl.fwd(*d_in, causal=w.causal)
+            h_L.copy_(Lx.detach(), non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        ke = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * fl_step * ke / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / ke, "api": "attention_kl_distillation_b200.streamkl"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, phase, args.cpu_seconds)
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) teacher, student = teacher + noise; bf16)",
+        "config": {**workload_desc(w, phase),
+                   "parallelism": f"dp{world} (independent replicas, no collective)"},
+        "pct_of_peak": value / world / peak,
+        "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac_of_peak": fwd_tf / peak,
+                "rows_per_s": w.BH * w.NQ / (fwd_ms * 1e-3)},
+        "bwd": ({"ms": bwd_ms, "tflops": bwd_tf, "frac_of_peak": bwd_tf / peak}
+                if bwd_tf else None),
+        "roofline": roofline,
+        "mufu_ceiling_frac_of_clock_peak": (w.d1 + w.d2) / 512,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -124,6 +124,13 @@ streamkl_status streamkl_set_wait_limit_ms(int ms);
 /* Version of this ABI: 1. */
 int streamkl_abi_version(void);
 
+/*
+ * Number of kernels this library has launched successfully in this process
+ * (all devices, all entry points).  Lets a caller count the device work a
+ * sequence of calls issued.
+ */
+uint64_t streamkl_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

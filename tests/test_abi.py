@@ -61,8 +61,8 @@ def test_fwd_rejects_nonfinite_scale():
 
 def test_workspace_size():
     ws = B.workspace_size(2, 3, 100, 50, 128, 64)
-    need = 2 * 3 * 100 * (128 + 64) * 4
-    assert ws >= need and ws % 256 == 0 and ws - need < 256 + 4096
+    need = 2 * 3 * 100 * (128 + 64) * 4 + 2 * 3 * 128 * 8 * 4   # dQ accumulator + row records
+    assert ws >= need and ws % 256 == 0 and ws - need <= 768
     assert B.workspace_size(1, 1, 0, 5, 64, 64) == 0
     assert B.workspace_size(1, 1, 5, 5, 96, 64) == 0
 
@@ -71,3 +71,38 @@ def test_wait_limit_validation():
     with pytest.raises(B.StreamKLError):
         B.set_wait_limit_ms(0)
     B.set_wait_limit_ms(2000)
+
+
+def _bwd_raw(prob, dL=256, ins=(16, 32, 48, 64), vecs=(512, 768, 1024), outs=(2048, 4096, 0, 0),
+             ws=1 << 20, ws_bytes=1 << 40):
+    lib = B.lib()
+    v = ctypes.c_void_p
+    return lib.streamkl_bwd(ctypes.byref(prob), v(dL), *[v(p) for p in ins], *[v(p) for p in vecs],
+                            *[v(p) for p in outs], v(ws), ctypes.c_size_t(ws_bytes), v(0))
+
+
+def test_bwd_rejects_bad_arguments():
+    prob = B.problem(1, 2, 100, 100, 128, 64, causal=True)
+    assert _bwd_raw(prob, dL=0) == B.EINVAL                          # missing dL
+    assert _bwd_raw(prob, ins=(16, 32, 0, 64)) == B.EINVAL            # missing input
+    assert _bwd_raw(prob, vecs=(512, 770, 1024)) == B.EINVAL          # misaligned LSE1
+    assert _bwd_raw(prob, outs=(0, 0, 0, 0)) == B.EINVAL              # nothing requested
+    assert _bwd_raw(prob, outs=(2056, 0, 0, 0)) == B.EINVAL           # misaligned output
+    assert _bwd_raw(prob, ws=0) == B.EINVAL                           # no workspace
+    assert _bwd_raw(prob, ws=(1 << 20) + 16) == B.EINVAL              # workspace not 256-aligned
+    need = B.workspace_size(1, 2, 100, 100, 128, 64, True)
+    assert _bwd_raw(prob, ws_bytes=need - 1) == B.EINVAL              # workspace too small
+    assert _bwd_raw(B.problem(1, 2, 100, 100, 96, 64)) == B.EUNSUPPORTED
+    assert _bwd_raw(B.problem(1, 2, 101, 100, 64, 64, causal=True)) == B.EINVAL
+
+
+def test_binding_argtypes_match_header():
+    """Each ctypes prototype has as many arguments as the header declares."""
+    import re
+    text = B.HEADER.read_text()
+    for name in B.header_functions():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", text)
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        fn = getattr(B.lib(), name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == len(params), name

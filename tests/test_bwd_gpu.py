@@ -1,0 +1,143 @@
+"""GPU parity of the backward (streamkl_bwd through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import TOL_GRAD, cuda_inputs, oracle_bits, rel_frobenius, workload
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [  # B, H, NQ, NK, d1, d2, causal
+    (1, 1, 64, 128, 64, 64, False),
+    (1, 2, 130, 200, 128, 128, True),
+    (1, 1, 100, 300, 128, 64, True),
+    (1, 1, 257, 257, 64, 128, False),
+    (2, 1, 1, 1, 128, 128, True),
+    (1, 1, 200, 100, 64, 64, False),
+    (1, 2, 384, 384, 128, 128, True),
+    (3, 2, 70, 333, 64, 64, True),
+]
+
+
+def run_bwd(dev, dL, causal, need=(True, True, True, True), s1=None, s2=None):
+    from attention_kl_distillation_b200 import bwd, fwd, query_device_status
+    L, A, B = fwd(*dev, causal=causal, s1=s1, s2=s2)
+    grads = bwd(dL, *dev, L, A, B, causal=causal, s1=s1, s2=s2, need=need)
+    torch.cuda.synchronize()
+    assert query_device_status() == 0
+    return [g.float().cpu().numpy().astype(np.float64) if g is not None else None for g in grads]
+
+
+def oracle_heads(orc, ins, dL, causal, heads, s1=None, s2=None):
+    B, H, NQ = dL.shape
+    g = dL.reshape(B * H, NQ).cpu().numpy().astype(np.float64)[heads]
+    return orc.bwd_heads(*oracle_bits(ins), heads, g, causal=causal, s1=s1, s2=s2)
+
+
+def check_grads(gpu, ora, heads, names=("dQ1", "dK1", "dQ2", "dK2"), what=""):
+    for n, gval in zip(("dQ1", "dK1", "dQ2", "dK2"), gpu):
+        if n not in names:
+            continue
+        G = gval.reshape(-1, *gval.shape[2:])[heads]
+        assert np.all(np.isfinite(G)), f"{what} {n} not finite"
+        if np.linalg.norm(ora[n]) == 0.0:
+            # e.g. a single visible key: the exact gradient vanishes; allow fp32 rounding residue
+            assert np.abs(G).max() <= 1e-6, f"{what} {n}: expected 0, max |g| {np.abs(G).max():.2e}"
+            continue
+        err = rel_frobenius(G, ora[n])
+        assert err <= TOL_GRAD, f"{what} {n}: relative Frobenius error {err:.3e}"
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B{}H{}Q{}K{}d{}-{}{}".format(*s[:6], "c" if s[6] else ""))
+def test_bwd_small_shapes(orc, shape):
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(*shape)
+    ins = make_inputs(w)
+    dL = torch.randn((w.B, w.H, w.NQ), generator=torch.Generator().manual_seed(11))
+    gpu = run_bwd(cuda_inputs(ins), dL.cuda(), w.causal)
+    heads = list(range(w.BH))
+    check_grads(gpu, oracle_heads(orc, ins, dL, w.causal, heads), heads, what=w.name)
+
+
+@pytest.mark.parametrize("config", ["teacher_fixed", "student_fixed"])
+def test_bwd_gradient_configurations(orc, config):
+    """NULL outputs skip work: teacher fixed returns only dQ2/dK2, student fixed only dQ1/dK1."""
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(1, 2, 192, 256, 128, 128, True)
+    ins = make_inputs(w)
+    dL = torch.randn((w.B, w.H, w.NQ), generator=torch.Generator().manual_seed(12))
+    need = (False, False, True, True) if config == "teacher_fixed" else (True, True, False, False)
+    gpu = run_bwd(cuda_inputs(ins), dL.cuda(), True, need=need)
+    assert [g is None for g in gpu] == [not x for x in need]
+    names = [n for n, x in zip(("dQ1", "dK1", "dQ2", "dK2"), need) if x]
+    check_grads(gpu, oracle_heads(orc, ins, dL, True, [0, 1]), [0, 1], names=names)
+
+
+def test_bwd_single_output(orc):
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(1, 1, 150, 150, 64, 128, False)
+    ins = make_inputs(w)
+    dL = torch.randn((1, 1, 150), generator=torch.Generator().manual_seed(13))
+    gpu = run_bwd(cuda_inputs(ins), dL.cuda(), False, need=(False, True, False, False))
+    check_grads(gpu, oracle_heads(orc, ins, dL, False, [0]), [0], names=["dK1"])
+
+
+def test_bwd_explicit_scales(orc):
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(1, 1, 128, 192, 128, 128, True)
+    ins = make_inputs(w)
+    dL = torch.randn((1, 1, 128), generator=torch.Generator().manual_seed(14))
+    gpu = run_bwd(cuda_inputs(ins), dL.cuda(), True, s1=0.2, s2=0.11)
+    check_grads(gpu, oracle_heads(orc, ins, dL, True, [0], s1=0.2, s2=0.11), [0])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_identical_inputs_give_exact_zero(causal):
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(1, 2, 200, 200, 128, 128, causal)
+    Q, K, _, _ = cuda_inputs(make_inputs(w))
+    dL = torch.randn((1, 2, 200), device="cuda")
+    for g in run_bwd([Q, K, Q, K], dL, causal):
+        assert np.all(g == 0.0)
+
+
+def test_autograd_wrapper_matches_direct_call():
+    from attention_kl_distillation_b200 import bwd, fwd, streamkl
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(1, 2, 130, 260, 128, 64, True)
+    Q1, K1, Q2, K2 = cuda_inputs(make_inputs(w))
+    ins = [t.clone().requires_grad_(True) for t in (Q1, K1, Q2, K2)]
+    L = streamkl(*ins, causal=True)
+    (L * 0.5).sum().backward()
+    L0, A, B = fwd(Q1, K1, Q2, K2, causal=True)
+    dL = torch.full_like(L0, 0.5)
+    ref = bwd(dL, Q1, K1, Q2, K2, L0, A, B, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(L.detach(), L0)
+    for t, r in zip(ins, ref):
+        err = ((t.grad.float() - r.float()).norm() / r.float().norm()).item()
+        assert err <= 1e-2   # fp32 atomics: not bitwise reproducible
+
+
+def test_bwd_full_size_workload(orc):
+    """Forward+backward workload (B1 H32 N16384 d128 causal, dL = 1/(B*H*NQ)):
+    dQ on >= 256 sampled rows of every head, dK1/dK2 in full on head 0 and one seeded head."""
+    from attention_kl_distillation_b200.inputs import WORKLOADS, make_inputs, sample_rows
+    w = WORKLOADS["fwdbwd16k"]
+    ins = make_inputs(w)
+    dev = cuda_inputs(ins)
+    g = 1.0 / (w.B * w.H * w.NQ)
+    dL = torch.full((w.B, w.H, w.NQ), g, device="cuda")
+    dQ1, dK1, dQ2, dK2 = run_bwd(dev, dL, True)
+    bits = oracle_bits(ins)
+    rows = sample_rows(w.BH, w.NQ, 256, seed=w.seed)
+    _, _, _, oq1, oq2 = orc.bwd_rows(*bits, rows, np.full(len(rows), g), causal=True)
+    gq1 = dQ1.reshape(w.BH, w.NQ, -1)[rows[:, 0], rows[:, 1]]
+    gq2 = dQ2.reshape(w.BH, w.NQ, -1)[rows[:, 0], rows[:, 1]]
+    assert rel_frobenius(gq1, oq1) <= TOL_GRAD
+    assert rel_frobenius(gq2, oq2) <= TOL_GRAD
+    heads = [0, int(np.random.default_rng(w.seed).integers(1, w.BH))]
+    o = orc.bwd_heads(*bits, heads, np.full((2, w.NQ), g), causal=True)
+    for n, G in (("dK1", dK1), ("dK2", dK2)):
+        err = rel_frobenius(G.reshape(w.BH, w.NK, -1)[heads], o[n])
+        assert err <= TOL_GRAD, f"{n} {err:.3e}"
