@@ -42,6 +42,8 @@ _lib.streamkl_bwd_workspace_size.argtypes = [_pp]
 _lib.streamkl_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.streamkl_bwd.argtypes = [_pp] + [_vp] * 13 + [ctypes.c_size_t, _vp]
 _lib.streamkl_bwd.restype = ctypes.c_int
+_lib.streamkl_bwd_noalloc.argtypes = [_pp] + [_vp] * 13
+_lib.streamkl_bwd_noalloc.restype = ctypes.c_int
 _lib.streamkl_status_string.argtypes = [ctypes.c_int]
 _lib.streamkl_status_string.restype = ctypes.c_char_p
 _lib.streamkl_query_device_status.argtypes = [_vp]
@@ -171,6 +173,24 @@ def bwd(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, causal=False, s1=None, s2=None,
     if st != OK:
         raise StreamKLError(st, "streamkl_bwd")
     return tuple(outs)
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def bwd_noalloc(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, out, causal=False, s1=None, s2=None):
+    """streamkl_bwd_noalloc: the backward without a caller workspace, for callers that
+    cannot allocate device memory.  ``out`` holds preallocated bf16 gradients (None skips
+    one); the library's own static scratch (64 MiB per GPU) replaces the workspace."""
+    B, H, NQ, NK, d1, d2 = _check_qk(Q1, K1, Q2, K2)
+    prob = problem(B, H, NQ, NK, d1, d2, causal, s1, s2)
+    with torch.cuda.device(Q1.device):
+        st = _lib.streamkl_bwd_noalloc(ctypes.byref(prob), _ptr(dL), _ptr(Q1), _ptr(K1), _ptr(Q2),
+                                       _ptr(K2), _ptr(L), _ptr(LSE1), _ptr(LSE2), *map(_ptr, out),
+                                       _stream(Q1.device))
+    if st != OK:
+        raise StreamKLError(st, "streamkl_bwd_noalloc")
+    return tuple(out)
 
 
 class _StreamKLFunction(torch.autograd.Function):

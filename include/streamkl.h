@@ -104,6 +104,37 @@ streamkl_status streamkl_bwd(const streamkl_problem *prob, const float *dL, cons
                              const float *LSE1, const float *LSE2, void *dQ1, void *dK1, void *dQ2,
                              void *dK2, void *workspace, size_t ws_bytes, streamkl_stream_t stream);
 
+/*
+ * Device scratch owned by streamkl_bwd_noalloc: 64 MiB, reserved on every GPU
+ * that loads this library and held until the process exits.
+ */
+#define STREAMKL_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * Backward for callers that cannot allocate device memory (the paper has no
+ * counterpart; it is an interface convenience).  Such callers include a
+ * framework whose caching allocator already holds the free device memory, or
+ * code that must not call cudaMalloc/cudaFree because those may synchronise
+ * the device.  Same arguments, results and errors as streamkl_bwd, without
+ * the workspace: the library uses its own static device scratch instead and
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - Problems whose streamkl_bwd_workspace_size exceeds
+ *    STREAMKL_NOALLOC_SCRATCH_BYTES are rejected with STREAMKL_EINVAL before
+ *    any CUDA call.
+ *  - The first call on a device looks up the scratch's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one scratch array, which keeps the
+ *    last call's contents (each call clears what must start at zero).  Calls
+ *    that overlap on the GPU (different streams, or threads without ordering)
+ *    race on it and give wrong gradients: order them on one stream.
+ */
+streamkl_status streamkl_bwd_noalloc(const streamkl_problem *prob, const float *dL,
+                                     const void *Q1, const void *K1, const void *Q2,
+                                     const void *K2, const float *L, const float *LSE1,
+                                     const float *LSE2, void *dQ1, void *dK1, void *dQ2,
+                                     void *dK2, streamkl_stream_t stream);
+
 /* Static English text for a status code. */
 const char *streamkl_status_string(streamkl_status st);
 
