@@ -20,12 +20,15 @@
 //                 dQ_t^T = K_t^T dS_t^T                     (M=d_t, N=64 queries)
 //               S for step t+1 is issued before the contractions of step t so
 //               that the tensor pipe works while dS is being formed.
-//   warps 2..5  dS warpgroup: thread j owns key j (TMEM lane j): loads its S1^T,
-//               S2^T rows, regenerates P1, P2 with exp2 on the MUFU pipe,
-//               forms s1*dS1 and s2*dS2 in bf16 and writes them once to shared
-//               memory in the 128B-swizzled layout that serves both as the
-//               K-major A operand of dK and the MN-major B operand of dQ^T.
-//   warps 6..9  dQ warpgroup: reads dQ^T (thread = feature index) and adds it
+//   warps 2..9  two dS warpgroups, for queries 0..31 and 32..63 of a step:
+//               thread j owns key j (TMEM lane j), loads its S1^T and S2^T
+//               row segments, regenerates P1, P2 with exp2 on the MUFU pipe
+//               (packed f32x2 arithmetic elsewhere), forms s1*dS1 and s2*dS2
+//               in bf16 and writes them once to shared memory in the
+//               128B-swizzled layout that serves both as the K-major A operand
+//               of dK and the MN-major B operand of dQ^T.  Two warpgroups put
+//               two dS warps on every SM sub-partition.
+//   warps 10..13 dQ warpgroup: reads dQ^T (thread = feature index) and adds it
 //               into the fp32 workspace with coalesced reductions; at the end
 //               of a unit converts the dK accumulators to bf16 and stores them.
 // TMEM (512 columns): S1^T [0,64) S2^T [64,128) dK1 [128,128+d1) dK2 [..,+d2)
@@ -42,7 +45,8 @@ namespace {
 
 constexpr int BK = kBwdBK;  // keys per unit
 constexpr int BQ = kBwdBQ;  // queries per step
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 448;
+constexpr int HALF = BQ / 2;  // queries per dS warpgroup
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kColS1 = 0, kColS2 = 64, kColDK1 = 128, kColDQ1 = 384, kColDQ2 = 448;
 
@@ -62,9 +66,9 @@ struct BwdLayout {
   static constexpr int q_off = k2_off + k2_bytes;
   static constexpr int ds_off = q_off + QSTAGES * qstage_bytes;
   static constexpr int bar_off = ds_off + DSBUF * 2 * ds_bytes;
-  // kfull kempty qfull[Q] qempty[Q] sfull sempty dsfull[D] dsempty[D] dqfull dqempty dkfull
-  // dkempty ufull[2] uempty[2] drain
-  static constexpr int nbar = 2 + 2 * QSTAGES + 2 + 2 * DSBUF + 4 + 4 + 1;
+  // kfull kempty qfull[Q] qempty[Q] sfull sempty dsfull[D] dsempty[D] dqfull dqempty1
+  // dqempty2 dkfull dkempty ufull[2] uempty[2] drain
+  static constexpr int nbar = 2 + 2 * QSTAGES + 2 + 2 * DSBUF + 5 + 4 + 1;
   static constexpr int misc_off = bar_off + nbar * 8;
   static constexpr int total = misc_off + 32;
   static constexpr int alloc = total + 1024;
@@ -107,45 +111,74 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-// dS for one key row j and the 64 queries of a step; writes the bf16 rows of
-// s1*dS1^T and s2*dS2^T (128 B each) into the swizzled tiles.
+// dS for one key row and HALF queries of a step (pairs of queries at a time,
+// packed f32x2).  s1/s2: raw products <K_t[key], Q_t[q]> from TMEM; rr: the
+// step's field-major row records offset to this half; writes the bf16 row
+// segments of s1*dS1^T and s2*dS2^T (HALF * 2 bytes each) into the swizzled
+// tiles at 16-byte chunks c0 .. c0 + HALF/8 - 1 of the key's 128-byte row.
+//   u_t = log2 P_t = c_t S_t - LSE_t log2e
+//   dS1 = s1 dL P1 (ln2 (u1 - u2) - L),   dS2 = s2 dL (P2 - P1)
+// MASK: visible iff key < NK and (not causal or q >= thr), with thr the first
+// visible query index of this half for this key.
 template <bool MASK>
-__device__ __forceinline__ void form_ds(const uint32_t (&s1)[BQ], const uint32_t (&s2)[BQ],
-                                        const float* rr, float c1, float c2, int j, int key,
-                                        int q0, int NK, int causal, int off, uint32_t ds1_row,
+__device__ __forceinline__ void form_ds(const uint32_t (&s1)[HALF], const uint32_t (&s2)[HALF],
+                                        const float* rr, float c1, float c2, int j, int c0,
+                                        bool key_ok, int thr, uint32_t ds1_row,
                                         uint32_t ds2_row) {
+  const float2 C1 = make_float2(c1, c1), C2 = make_float2(c2, c2);
+  const float2 NEG1 = make_float2(-1.f, -1.f), LN2 = make_float2(kLn2, kLn2);
 #pragma unroll
-  for (int c = 0; c < BQ / 8; ++c) {
+  for (int c = 0; c < HALF / 8; ++c) {
     uint32_t w1[4], w2[4];
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      float d1v[2], d2v[2];
+    for (int h = 0; h < 2; ++h) {  // 4 queries per h
+      const int q = c * 8 + h * 4;
+      const float4 nb1 = *reinterpret_cast<const float4*>(rr + 0 * BQ + q);
+      const float4 nb2 = *reinterpret_cast<const float4*>(rr + 1 * BQ + q);
+      const float4 nL = *reinterpret_cast<const float4*>(rr + 2 * BQ + q);
+      const float4 g1 = *reinterpret_cast<const float4*>(rr + 3 * BQ + q);
+      const float4 g2 = *reinterpret_cast<const float4*>(rr + 4 * BQ + q);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int i = c * 8 + h * 2 + e;
-        const float4 r = *reinterpret_cast<const float4*>(rr + i * kRowRec);
-        const float g2 = rr[i * kRowRec + 4];
-        const float u1 = fmaf(__uint_as_float(s1[i]), c1, -r.x);
-        const float u2 = fmaf(__uint_as_float(s2[i]), c2, -r.y);
-        const float P1 = ex2(u1), P2 = ex2(u2);
-        const float t = fmaf(u1 - u2, kLn2, -r.z);
-        float a = r.w * (P1 * t);
-        float b = g2 * (P2 - P1);
+      for (int e = 0; e < 2; ++e) {  // a pair of queries
+        const int i = q + 2 * e;
+        const float2 S1 = make_float2(__uint_as_float(s1[i]), __uint_as_float(s1[i + 1]));
+        const float2 S2 = make_float2(__uint_as_float(s2[i]), __uint_as_float(s2[i + 1]));
+        const float2 B1 = e ? make_float2(nb1.z, nb1.w) : make_float2(nb1.x, nb1.y);
+        const float2 B2 = e ? make_float2(nb2.z, nb2.w) : make_float2(nb2.x, nb2.y);
+        const float2 NL = e ? make_float2(nL.z, nL.w) : make_float2(nL.x, nL.y);
+        const float2 G1 = e ? make_float2(g1.z, g1.w) : make_float2(g1.x, g1.y);
+        const float2 G2 = e ? make_float2(g2.z, g2.w) : make_float2(g2.x, g2.y);
+        const float2 u1 = __ffma2_rn(S1, C1, B1);
+        const float2 u2 = __ffma2_rn(S2, C2, B2);
+        const float2 P1 = make_float2(ex2(u1.x), ex2(u1.y));
+        const float2 P2 = make_float2(ex2(u2.x), ex2(u2.y));
+        const float2 t = __ffma2_rn(__ffma2_rn(u2, NEG1, u1), LN2, NL);
+        float2 d1 = __fmul2_rn(__fmul2_rn(P1, t), G1);
+        float2 d2 = __fmul2_rn(__ffma2_rn(P1, NEG1, P2), G2);
         if (MASK) {
-          const bool vis = key < NK && (!causal || key <= q0 + i + off);
-          a = vis ? a : 0.f;
-          b = vis ? b : 0.f;
+          const bool vx = key_ok && i >= thr, vy = key_ok && i + 1 >= thr;
+          d1.x = vx ? d1.x : 0.f;
+          d2.x = vx ? d2.x : 0.f;
+          d1.y = vy ? d1.y : 0.f;
+          d2.y = vy ? d2.y : 0.f;
         }
-        d1v[e] = a;
-        d2v[e] = b;
+        w1[h * 2 + e] = pack_bf16(d1.x, d1.y);
+        w2[h * 2 + e] = pack_bf16(d2.x, d2.y);
       }
-      w1[h] = pack_bf16(d1v[0], d1v[1]);
-      w2[h] = pack_bf16(d2v[0], d2v[1]);
     }
-    const uint32_t sw = static_cast<uint32_t>((c ^ (j & 7)) << 4);
+    const uint32_t sw = static_cast<uint32_t>(((c0 + c) ^ (j & 7)) << 4);
     st_shared_v4(ds1_row + sw, w1[0], w1[1], w1[2], w1[3]);
     st_shared_v4(ds2_row + sw, w2[0], w2[1], w2[2], w2[3]);
   }
+}
+
+// Adds one dQ_t^T column block (64 queries of feature f) into the fp32
+// accumulator: base points at row q0, feature f; rows are LDQ floats apart.
+template <int LDQ, bool FULL>
+__device__ __forceinline__ void red_dq(float* base, const uint32_t (&v)[BQ], int nvalid) {
+#pragma unroll
+  for (int i = 0; i < BQ; ++i)
+    if (FULL || i < nvalid) atomicAdd(base + i * LDQ, __uint_as_float(v[i]));
 }
 
 template <int D1, int D2>
@@ -153,6 +186,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
   using Lay = BwdLayout<D1, D2>;
   constexpr int QST = Lay::QSTAGES;
   constexpr int DSB = Lay::DSBUF;
+  constexpr int LDQ = D1 + D2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -166,8 +200,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
   uint64_t* dsfull = sempty + 1;
   uint64_t* dsempty = dsfull + DSB;
   uint64_t* dqfull = dsempty + DSB;
-  uint64_t* dqempty = dqfull + 1;
-  uint64_t* dkfull = dqempty + 1;
+  uint64_t* dqempty = dqfull + 1;  // [2]: dQ1^T and dQ2^T slots read out
+  uint64_t* dkfull = dqempty + 2;
   uint64_t* dkempty = dkfull + 1;
   uint64_t* ufull = dkempty + 1;
   uint64_t* uempty = ufull + 2;
@@ -189,18 +223,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       mbar_init(&qempty[s], 1);
     }
     mbar_init(sfull, 1);
-    mbar_init(sempty, 4);
+    mbar_init(sempty, 8);  // every warp of both dS warpgroups
     for (int s = 0; s < DSB; ++s) {
-      mbar_init(&dsfull[s], 4);
+      mbar_init(&dsfull[s], 8);
       mbar_init(&dsempty[s], 1);
     }
     mbar_init(dqfull, 1);
-    mbar_init(dqempty, 4);
+    mbar_init(&dqempty[0], 4);
+    mbar_init(&dqempty[1], 4);
     mbar_init(dkfull, 1);
     mbar_init(dkempty, 4);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ufull[s], 1);
-      mbar_init(&uempty[s], 9);  // MMA thread + 4 dS warps + 4 dQ warps
+      mbar_init(&uempty[s], 13);  // MMA thread + 8 dS warps + 4 dQ warps
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -302,7 +337,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       constexpr uint32_t idQ2 = idesc_bf16(D2, BQ, 1, 1);
       const uint32_t k1a = smem_u32(k1_s), k2a = smem_u32(k2_s);
       int us = 0, qs_s = 0, qs_r = 0, db = 0;
-      uint32_t uph = 0, kph = 0, qph_s = 0, sph = 0, dqph = 0, dkph = 0;
+      uint32_t uph = 0, kph = 0, qph_s = 0, sph = 0, dkph = 0;
+      uint32_t dqph[2] = {0, 0};
       uint32_t dsph[DSB] = {};
       bool ok = true;
       for (;;) {
@@ -353,8 +389,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
             if (!(ok = mbar_wait(dkempty, dkph ^ 1, ctl))) break;
             dkph ^= 1;
           }
-          if (!(ok = mbar_wait(dqempty, dqph ^ 1, ctl))) break;
-          dqph ^= 1;
           tc_fence_after();
           const uint32_t qa1 = smem_u32(q1_s(qs_r)), qa2 = smem_u32(q2_s(qs_r));
           const uint32_t d1a = smem_u32(ds1_s(db)), d2a = smem_u32(ds2_s(db));
@@ -371,12 +405,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           }
           // dQ_t^T = K_t^T (s_t dS_t)^T : A = K tile read MN-major (64-feature chunks
           // 16 KB apart), B = dS^T read MN-major (64 queries contiguous per key).
+          if (!(ok = mbar_wait(&dqempty[0], dqph[0] ^ 1, ctl))) break;
+          dqph[0] ^= 1;
+          tc_fence_after();
+          if (p.want_dq1) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            if (p.want_dq1)
+            for (int kk = 0; kk < BK / 16; ++kk)
               umma_bf16_ss(tmem_base + kColDQ1, sdesc_sw128(k1a + kk * 2048, BK * 128, 1024),
                            sdesc_sw128(d1a + kk * 2048, BQ * 128, 1024), idQ1, kk > 0);
-            if (p.want_dq2)
+          }
+          if (!(ok = mbar_wait(&dqempty[1], dqph[1] ^ 1, ctl))) break;
+          dqph[1] ^= 1;
+          tc_fence_after();
+          if (p.want_dq2) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
               umma_bf16_ss(tmem_base + kColDQ2, sdesc_sw128(k2a + kk * 2048, BK * 128, 1024),
                            sdesc_sw128(d2a + kk * 2048, BQ * 128, 1024), idQ2, kk > 0);
           }
@@ -395,8 +438,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
       mbar_wait(drain, 0, dctl);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ dS warpgroup
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ dS warpgroups
+    const int half = (warp - 2) >> 2;  // queries [half*32, half*32 + 32) of each step
     const int quarter = warp & 3;
     const int j = quarter * 32 + lane;  // key row within the tile
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -416,17 +460,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       if (u < 0) break;
       const UnitB w = decode_unit(p, u);
       const int key = w.k0 + j;
+      const bool key_ok = key < p.NK;
       for (int t = 0; t < w.nsteps; ++t) {
         const int q0 = (w.qt0 + t) * BQ;
-        if (!(ok = mbar_wait(&qfull[qs], qph, ctl))) break;  // per-row records of this step
+        if (!(ok = mbar_wait(&qfull[qs], qph, ctl))) break;  // row records of this step
         if (!(ok = mbar_wait(sfull, sph, ctl))) break;
         sph ^= 1;
         tc_fence_after();
-        uint32_t a[BQ], b[BQ];
-        tmem_ld_32x32b_x32(tl + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-        tmem_ld_32x32b_x32(tl + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-        tmem_ld_32x32b_x32(tl + kColS2, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
-        tmem_ld_32x32b_x32(tl + kColS2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
+        uint32_t a[HALF], b[HALF];
+        tmem_ld_32x32b_x32(tl + kColS1 + half * HALF, a);
+        tmem_ld_32x32b_x32(tl + kColS2 + half * HALF, b);
         tmem_ld_wait();
         reg_fence(a);
         reg_fence(b);
@@ -436,12 +479,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
         dsph[db] ^= 1;
         const uint32_t r1 = smem_u32(ds1_s(db)) + j * 128, r2 = smem_u32(ds2_s(db)) + j * 128;
-        const bool masked =
-            (p.causal && q0 + off < w.k0 + BK - 1) || (w.k0 + BK > p.NK);
-        if (masked)
-          form_ds<true>(a, b, rr_s(qs), p.c1, p.c2, j, key, q0, p.NK, p.causal, off, r1, r2);
-        else
-          form_ds<false>(a, b, rr_s(qs), p.c1, p.c2, j, key, q0, p.NK, p.causal, off, r1, r2);
+        const float* rr = rr_s(qs) + half * HALF;
+        const bool masked = (p.causal && q0 + off < w.k0 + BK - 1) || (w.k0 + BK > p.NK);
+        if (masked) {
+          // first visible query (index within this half) for this key
+          const int thr = p.causal ? key - off - q0 - half * HALF : -1;
+          form_ds<true>(a, b, rr, p.c1, p.c2, j, half * (HALF / 8), key_ok, thr, r1, r2);
+        } else {
+          form_ds<false>(a, b, rr, p.c1, p.c2, j, half * (HALF / 8), true, 0, r1, r2);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&dsfull[db]);
@@ -461,7 +507,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
     // features 16q..16q+15 in lanes 32q..32q+15.
     const int f1 = (D1 == 128) ? quarter * 32 + lane : (lane < 16 ? quarter * 16 + lane : -1);
     const int f2 = (D2 == 128) ? quarter * 32 + lane : (lane < 16 ? quarter * 16 + lane : -1);
-    const int ldq = D1 + D2;
     int us = 0;
     uint32_t uph = 0, dqph = 0, dkph = 0;
     bool ok = true;
@@ -481,33 +526,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         if (!(ok = mbar_wait(dqfull, dqph, ctl))) break;
         dqph ^= 1;
         tc_fence_after();
-        uint32_t a[BQ], b[BQ];
-        if (p.want_dq1) {
-          tmem_ld_32x32b_x32(tl + kColDQ1, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-          tmem_ld_32x32b_x32(tl + kColDQ1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-        }
-        if (p.want_dq2) {
-          tmem_ld_32x32b_x32(tl + kColDQ2, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
-          tmem_ld_32x32b_x32(tl + kColDQ2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
-        }
-        tmem_ld_wait();
-        reg_fence(a);
-        reg_fence(b);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dqempty);
         const int nvalid = min(BQ, p.NQ - q0);
-        float* base = p.dQacc + (static_cast<size_t>(w.bh) * p.NQ + q0) * ldq;
-        if (p.want_dq1 && f1 >= 0) {
+        float* base = p.dQacc + (static_cast<size_t>(w.bh) * p.NQ + q0) * LDQ;
 #pragma unroll
-          for (int i = 0; i < BQ; ++i)
-            if (i < nvalid) atomicAdd(base + static_cast<size_t>(i) * ldq + f1, __uint_as_float(a[i]));
-        }
-        if (p.want_dq2 && f2 >= 0) {
-#pragma unroll
-          for (int i = 0; i < BQ; ++i)
-            if (i < nvalid)
-              atomicAdd(base + static_cast<size_t>(i) * ldq + D1 + f2, __uint_as_float(b[i]));
+        for (int tsel = 0; tsel < 2; ++tsel) {
+          const bool want = tsel == 0 ? p.want_dq1 : p.want_dq2;
+          const int f = tsel == 0 ? f1 : D1 + f2;
+          const bool fok = (tsel == 0 ? f1 : f2) >= 0;
+          uint32_t v[BQ];
+          if (want) {
+            const uint32_t col = tl + (tsel == 0 ? kColDQ1 : kColDQ2);
+            tmem_ld_32x32b_x32(col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tmem_ld_32x32b_x32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tmem_ld_wait();
+            reg_fence(v);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dqempty[tsel]);
+          if (want && fok) {
+            if (nvalid == BQ)
+              red_dq<LDQ, true>(base + f, v, BQ);
+            else
+              red_dq<LDQ, false>(base + f, v, nvalid);
+          }
         }
       }
       if (!ok) break;
@@ -517,33 +559,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       tc_fence_after();
       const int key = w.k0 + quarter * 32 + lane;
       const bool row_ok = key < p.NK;
-      if (p.want_dk1) {
-        __nv_bfloat16* dst = p.dK1 + (static_cast<size_t>(w.bh) * p.NK + key) * D1;
 #pragma unroll
-        for (int c = 0; c < D1; c += 32) {
+      for (int tsel = 0; tsel < 2; ++tsel) {
+        const bool want = tsel == 0 ? p.want_dk1 : p.want_dk2;
+        if (!want) continue;
+        constexpr int DMAX = D1 > D2 ? D1 : D2;
+        const int D = tsel == 0 ? D1 : D2;
+        __nv_bfloat16* dst =
+            (tsel == 0 ? p.dK1 : p.dK2) + (static_cast<size_t>(w.bh) * p.NK + key) * D;
+        const uint32_t col0 = tl + kColDK1 + (tsel == 0 ? 0 : D1);
+#pragma unroll
+        for (int c = 0; c < DMAX; c += 32) {
+          if (c >= D) break;
           uint32_t v[32];
-          tmem_ld_32x32b_x32(tl + kColDK1 + c, v);
-          tmem_ld_wait();
-          reg_fence(v);
-          if (row_ok) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 o;
-              o.x = pack_bf16(__uint_as_float(v[e + 0]), __uint_as_float(v[e + 1]));
-              o.y = pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-              o.z = pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
-              o.w = pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
-              *reinterpret_cast<uint4*>(dst + c + e) = o;
-            }
-          }
-        }
-      }
-      if (p.want_dk2) {
-        __nv_bfloat16* dst = p.dK2 + (static_cast<size_t>(w.bh) * p.NK + key) * D2;
-#pragma unroll
-        for (int c = 0; c < D2; c += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tl + kColDK1 + D1 + c, v);
+          tmem_ld_32x32b_x32(col0 + c, v);
           tmem_ld_wait();
           reg_fence(v);
           if (row_ok) {
@@ -574,26 +603,33 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
   }
 }
 
-// Per-row records (LSE1*log2e, LSE2*log2e, L, s1*dL, s2*dL, 0, 0, 0) padded to
-// whole 64-row steps with zeros (zero weight makes padded rows contribute
-// nothing), the zeroed dQ accumulator and the unit counter.
+// Per-row records for the backward, field-major per 64-row step
+// ([bh][step][field][64]): -LSE1*log2e, -LSE2*log2e, -L, s1*dL, s2*dL, 0, 0, 0.
+// Rows past NQ (padding of the last step) get all zeros, so their weight is
+// zero and they contribute nothing.  Also zeroes the dQ accumulator and the
+// work-unit counter that follows the records.
 __global__ void streamkl_bwd_prep_kernel(const BwdPrepParams p) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long nrec = static_cast<long long>(p.BH) * p.NQpad;
   constexpr float kLog2e = 1.4426950408889634f;
+  constexpr int S = kBwdBQ;
   for (long long r = tid; r < nrec; r += stride) {
     const int bh = static_cast<int>(r / p.NQpad);
     const int i = static_cast<int>(r % p.NQpad);
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = make_float4(0.f, 0.f, 0.f, 0.f);
+    float f[kRowRec] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (i < p.NQ) {
       const size_t o = static_cast<size_t>(bh) * p.NQ + i;
       const float g = p.dL[o];
-      a = make_float4(p.LSE1[o] * kLog2e, p.LSE2[o] * kLog2e, p.L[o], p.s1 * g);
-      b.x = p.s2 * g;
+      f[0] = -p.LSE1[o] * kLog2e;
+      f[1] = -p.LSE2[o] * kLog2e;
+      f[2] = -p.L[o];
+      f[3] = p.s1 * g;
+      f[4] = p.s2 * g;
     }
-    reinterpret_cast<float4*>(p.rowrec)[2 * r] = a;
-    reinterpret_cast<float4*>(p.rowrec)[2 * r + 1] = b;
+    float* rec = p.rowrec + (static_cast<size_t>(bh) * p.NQpad + (i / S) * S) * kRowRec + (i % S);
+#pragma unroll
+    for (int k = 0; k < kRowRec; ++k) rec[k * S] = f[k];
   }
   const long long n4 = p.dqacc_elems / 4;
   for (long long e = tid; e < n4; e += stride)

@@ -6,21 +6,28 @@
 // Key tiles past the causal frontier are never loaded or multiplied.
 //
 // B200 mapping (one CTA per SM, persistent):
-//   warp 0      TMA producer: Q1/Q2 tile once per work unit, K1/K2 tiles into
-//               a 4-stage shared-memory ring (128-byte swizzle, no multicast).
-//   warp 1      TMEM owner and UMMA issuer: S1 = Q1 K1^T and S2 = Q2 K2^T for
-//               each key tile (tcgen05.mma kind::f16, fp32 accumulators) into
-//               one of four TMEM buffers of 2 x 64 columns.
-//   warps 2..5  reduction warpgroup: thread r owns query row r (TMEM lane r),
-//               loads its 64 + 64 logits with tcgen05.ld, frees the buffer and
-//               applies the online update in registers (exp2 on the MUFU pipe,
-//               softmax scale folded into the exponent argument).
+//   work unit   (bh, 256-row query block) = two 128-row tiles A and B that
+//               share every key tile, so each K tile is read once per 256 rows
+//   warp 0      TMA producer: Q1/Q2 for both tiles once per unit, K1/K2 tiles
+//               into a shared-memory ring (128-byte swizzle, no multicast)
+//   warp 1      TMEM owner and UMMA issuer: per key tile and query tile,
+//               S1 = Q1 K1^T and S2 = Q2 K2^T (tcgen05.mma kind::f16, fp32
+//               accumulators) into that tile's double-buffered TMEM slot
+//   warps 2..5  reduction warpgroup of tile A, warps 6..9 of tile B: thread r
+//               owns query row r (TMEM lane r), loads its 64 + 64 logits with
+//               tcgen05.ld, frees the slot and applies the online update in
+//               registers: exp2 on the MUFU pipe, the softmax scale folded into
+//               the exponent argument, packed f32x2 arithmetic elsewhere.
+//               Two warpgroups put two reduction warps on every SM sub-partition
+//               so that one hides the other's latencies.
 // The accumulator acc is one fp32 per row: there is no PV product and no
-// output tile, which is what lets both S tiles live in TMEM at once.
+// output tile, which is what lets both S tiles of both query tiles live in
+// TMEM (4 x 128 of the 512 columns) at once.
 //
-// Work units are (bh, 128-row query tile), visited longest first (the last
-// query tiles of a causal problem see the most keys) and dealt to CTAs in a
-// snake order, an approximation of longest-processing-time scheduling.
+// Units are visited longest first (the last query blocks of a causal problem
+// see the most keys) and dealt to CTAs in a snake order, an approximation of
+// longest-processing-time scheduling; units of one query block across heads
+// run together, so they stream the same key range through L2.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -30,29 +37,32 @@ namespace skl {
 namespace {
 
 constexpr int BQ = kFwdBQ;
+constexpr int NT = kFwdTiles;
 constexpr int BK = kFwdBK;
-constexpr int KSTAGES = 4;            // K1/K2 shared-memory ring depth
-constexpr int SBUF = 512 / (2 * BK);  // TMEM S1/S2 buffers (4 x 128 columns)
-constexpr int NTHREADS = 192;
+constexpr int SBUF = 2;  // TMEM S1/S2 slots per query tile
+constexpr int NTHREADS = 64 + NT * 128;
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D1, int D2>
 struct FwdLayout {
-  static constexpr int q1_bytes = BQ * D1 * 2;
-  static constexpr int q2_bytes = BQ * D2 * 2;
+  static constexpr int q1_tile = BQ * D1 * 2;
+  static constexpr int q2_tile = BQ * D2 * 2;
   static constexpr int k1_bytes = BK * D1 * 2;
   static constexpr int k2_bytes = BK * D2 * 2;
   static constexpr int stage_bytes = k1_bytes + k2_bytes;
+  static constexpr int q_bytes = NT * (q1_tile + q2_tile);
+  static constexpr int KSTAGES = (q_bytes + 4 * stage_bytes + 2048 <= 232448) ? 4 : 3;
   static constexpr int q1_off = 0;
-  static constexpr int q2_off = q1_off + q1_bytes;
-  static constexpr int k_off = q2_off + q2_bytes;
+  static constexpr int q2_off = q1_off + NT * q1_tile;
+  static constexpr int k_off = q2_off + NT * q2_tile;
   static constexpr int bar_off = k_off + KSTAGES * stage_bytes;
-  // barriers: qfull, qempty, kfull[KSTAGES], kempty[KSTAGES], sfull[SBUF], sempty[SBUF], drain
-  static constexpr int nbar = 3 + 2 * KSTAGES + 2 * SBUF;
+  // barriers: qfull, qempty, kfull[KS], kempty[KS], sfull[NT][SBUF], sempty[NT][SBUF], drain
+  static constexpr int nbar = 3 + 2 * KSTAGES + 2 * NT * SBUF;
   static constexpr int misc_off = bar_off + nbar * 8;
   static constexpr int total = misc_off + 16;
   static constexpr int alloc = total + 1024;  // slack to align the base to 1024 B
-  static_assert(q1_bytes % 1024 == 0 && q2_bytes % 1024 == 0 && k1_bytes % 1024 == 0 &&
+  static_assert(alloc <= 232448, "shared memory budget exceeded");
+  static_assert(q1_tile % 1024 == 0 && q2_tile % 1024 == 0 && k1_bytes % 1024 == 0 &&
                     k2_bytes % 1024 == 0,
                 "tiles must keep 1024-byte alignment for the 128B swizzle atoms");
 };
@@ -74,26 +84,36 @@ struct Sched {
 };
 
 struct Unit {
-  int bh, q0, nkt, kt_mask;  // key tiles [kt_mask, nkt) need element masks
+  int bh, q0;
+  int nkt[NT];     // key tiles each query tile needs (0: tile holds no valid row)
+  int kt_mask[NT]; // key tiles [kt_mask, nkt) need element masks
+  int nkt_max;
 };
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
-  const int nqt = (p.NQ + BQ - 1) / BQ;
+  const int nqb = (p.NQ + BQ * NT - 1) / (BQ * NT);
   Unit w;
   w.bh = u % p.BH;
-  const int qt = nqt - 1 - u / p.BH;  // longest (last) query tiles first
-  w.q0 = qt * BQ;
+  w.q0 = (nqb - 1 - u / p.BH) * (BQ * NT);  // longest (last) query blocks first
   const int nkt_all = (p.NK + BK - 1) / BK;
+  const int tail = (p.NK % BK) ? nkt_all - 1 : nkt_all;
   const int off = p.NK - p.NQ;
-  int nkt = nkt_all;
-  int kt_mask = (p.NK % BK) ? nkt_all - 1 : nkt_all;
-  if (p.causal) {
-    const int last = min(w.q0 + BQ - 1, p.NQ - 1) + off;  // last key any row of the tile sees
-    nkt = min(nkt_all, last / BK + 1);
-    kt_mask = min(kt_mask, (w.q0 + off + 1) / BK);  // first tile the first row cannot fully see
+  w.nkt_max = 0;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int r0 = w.q0 + t * BQ;
+    int nkt = nkt_all, km = tail;
+    if (r0 >= p.NQ) {
+      nkt = 0;
+    } else if (p.causal) {
+      const int last = min(r0 + BQ - 1, p.NQ - 1) + off;  // last key any row of the tile sees
+      nkt = min(nkt_all, last / BK + 1);
+      km = min(km, (r0 + off + 1) / BK);  // first tile the first row cannot fully see
+    }
+    w.nkt[t] = nkt;
+    w.kt_mask[t] = km;
+    w.nkt_max = max(w.nkt_max, nkt);
   }
-  w.nkt = nkt;
-  w.kt_mask = kt_mask;
   return w;
 }
 
@@ -111,40 +131,51 @@ __device__ __forceinline__ void tile_update(const uint32_t (&a)[BK], const uint3
 #pragma unroll
   for (int k = 0; k < 4; ++k) mx1[k] = mx2[k] = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < BK; ++j) {
-    float v1 = __uint_as_float(a[j]), v2 = __uint_as_float(b[j]);
-    if (MASK && j >= nv) v1 = v2 = -INFINITY;
-    mx1[j & 3] = fmaxf(mx1[j & 3], v1);
-    mx2[j & 3] = fmaxf(mx2[j & 3], v2);
+  for (int j = 0; j < BK; j += 2) {
+    float v1a = __uint_as_float(a[j]), v1b = __uint_as_float(a[j + 1]);
+    float v2a = __uint_as_float(b[j]), v2b = __uint_as_float(b[j + 1]);
+    if (MASK) {
+      if (j >= nv) v1a = v2a = -INFINITY;
+      if (j + 1 >= nv) v1b = v2b = -INFINITY;
+    }
+    const int k = (j >> 1) & 3;
+    mx1[k] = max3(mx1[k], v1a, v1b);
+    mx2[k] = max3(mx2[k], v2a, v2b);
   }
-  const float tmx1 = fmaxf(fmaxf(mx1[0], mx1[1]), fmaxf(mx1[2], mx1[3]));
-  const float tmx2 = fmaxf(fmaxf(mx2[0], mx2[1]), fmaxf(mx2[2], mx2[3]));
+  const float tmx1 = fmaxf(max3(mx1[0], mx1[1], mx1[2]), mx1[3]);
+  const float tmx2 = fmaxf(max3(mx2[0], mx2[1], mx2[2]), mx2[3]);
   const float m1n = fmaxf(st.m1, tmx1 * c1);
   const float m2n = fmaxf(st.m2, tmx2 * c2);
   // A row that has seen no key yet keeps m = -inf; shift by 0 instead so that
   // no inf - inf appears.  (Every valid row sees key 0 in its first tile.)
   const float m1u = (m1n == -INFINITY) ? 0.f : m1n;
   const float m2u = (m2n == -INFINITY) ? 0.f : m2n;
-  float sp1[4], sp2[4], sd[4];
+  const float2 C1 = make_float2(c1, c1), C2 = make_float2(c2, c2);
+  const float2 M1 = make_float2(-m1u, -m1u), M2 = make_float2(-m2u, -m2u);
+  const float2 NEG1 = make_float2(-1.f, -1.f);
+  float2 sp1[2], sp2[2], sd[2];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) sp1[k] = sp2[k] = sd[k] = 0.f;
+  for (int k = 0; k < 2; ++k) sp1[k] = sp2[k] = sd[k] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int j = 0; j < BK; ++j) {
-    float t1 = fmaf(__uint_as_float(a[j]), c1, -m1u);
-    float t2 = fmaf(__uint_as_float(b[j]), c2, -m2u);
-    float p1 = ex2(t1), p2 = ex2(t2);
-    if (MASK && j >= nv) {
-      p1 = 0.f;
-      p2 = 0.f;
-      t1 = t2 = 0.f;
+  for (int j = 0; j < BK; j += 2) {
+    const float2 v1 = make_float2(__uint_as_float(a[j]), __uint_as_float(a[j + 1]));
+    const float2 v2 = make_float2(__uint_as_float(b[j]), __uint_as_float(b[j + 1]));
+    float2 t1 = __ffma2_rn(v1, C1, M1);  // log2 of the unnormalised teacher weight
+    float2 t2 = __ffma2_rn(v2, C2, M2);
+    float2 p1 = make_float2(ex2(t1.x), ex2(t1.y));
+    float2 p2 = make_float2(ex2(t2.x), ex2(t2.y));
+    if (MASK) {
+      if (j >= nv) p1.x = p2.x = t1.x = t2.x = 0.f;
+      if (j + 1 >= nv) p1.y = p2.y = t1.y = t2.y = 0.f;
     }
-    sp1[j & 3] += p1;
-    sp2[j & 3] += p2;
-    sd[j & 3] = fmaf(p1, t1 - t2, sd[j & 3]);
+    const int k = (j >> 1) & 1;
+    sp1[k] = __fadd2_rn(sp1[k], p1);
+    sp2[k] = __fadd2_rn(sp2[k], p2);
+    sd[k] = __ffma2_rn(p1, __ffma2_rn(t2, NEG1, t1), sd[k]);  // p1 * (t1 - t2)
   }
-  const float s1 = (sp1[0] + sp1[1]) + (sp1[2] + sp1[3]);
-  const float s2 = (sp2[0] + sp2[1]) + (sp2[2] + sp2[3]);
-  const float d = (sd[0] + sd[1]) + (sd[2] + sd[3]);
+  const float s1 = (sp1[0].x + sp1[0].y) + (sp1[1].x + sp1[1].y);
+  const float s2 = (sp2[0].x + sp2[0].y) + (sp2[1].x + sp2[1].y);
+  const float d = (sd[0].x + sd[0].y) + (sd[1].x + sd[1].y);
   const float a1 = ex2(((st.m1 == -INFINITY) ? m1u : st.m1) - m1u);
   const float a2 = ex2(((st.m2 == -INFINITY) ? m2u : st.m2) - m2u);
   // sum_j p1 (y1 - y2) with y1 - y2 = (t1 - t2) + (m1 - m2)
@@ -158,6 +189,7 @@ __device__ __forceinline__ void tile_update(const uint32_t (&a)[BK], const uint3
 template <int D1, int D2>
 __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_constant__ FwdParams p) {
   using Lay = FwdLayout<D1, D2>;
+  constexpr int KS = Lay::KSTAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -165,10 +197,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
   uint64_t* qfull = bars + 0;
   uint64_t* qempty = bars + 1;
   uint64_t* kfull = bars + 2;
-  uint64_t* kempty = kfull + KSTAGES;
-  uint64_t* sfull = kempty + KSTAGES;
-  uint64_t* sempty = sfull + SBUF;
-  uint64_t* drain = sempty + SBUF;
+  uint64_t* kempty = kfull + KS;
+  uint64_t* sfull = kempty + KS;      // [NT][SBUF]
+  uint64_t* sempty = sfull + NT * SBUF;
+  uint64_t* drain = sempty + NT * SBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::misc_off + 4);
 
@@ -180,13 +212,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     *abort_flag = 0;
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
-    for (int s = 0; s < KSTAGES; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(&kfull[s], 1);
       mbar_init(&kempty[s], 1);
     }
-    for (int s = 0; s < SBUF; ++s) {
+    for (int s = 0; s < NT * SBUF; ++s) {
       mbar_init(&sfull[s], 1);
-      mbar_init(&sempty[s], 4);  // one arrival per reduction warp
+      mbar_init(&sempty[s], 4);  // one arrival per reduction warp of that tile
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -205,8 +237,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
   const uint32_t tmem_base = *tmem_slot;
 
   Sched sched{fwd_units(p.BH, p.NQ), static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x), 0};
-  uint8_t* q1_s = smem + Lay::q1_off;
-  uint8_t* q2_s = smem + Lay::q2_off;
+  auto q1_s = [&](int t) { return smem + Lay::q1_off + t * Lay::q1_tile; };
+  auto q2_s = [&](int t) { return smem + Lay::q2_off + t * Lay::q2_tile; };
   auto k1_s = [&](int s) { return smem + Lay::k_off + s * Lay::stage_bytes; };
   auto k2_s = [&](int s) { return smem + Lay::k_off + s * Lay::stage_bytes + Lay::k1_bytes; };
 
@@ -215,22 +247,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     if (lane == 0) {
       int ks = 0;
       uint32_t kph = 0, qph = 0;
-      uint32_t armed_q = 0, armed_k[KSTAGES] = {};  // last armed phase + 1 (0 = never)
+      uint32_t armed_q = 0, armed_k[KS] = {};  // last armed phase + 1 (0 = never)
       int u;
       bool ok = true;
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
         if (!(ok = mbar_wait(qempty, qph ^ 1, ctl))) break;
-        mbar_arrive_expect_tx(qfull, Lay::q1_bytes + Lay::q2_bytes);
+        mbar_arrive_expect_tx(qfull, Lay::q_bytes);
 #pragma unroll
-        for (int b = 0; b < D1 / 64; ++b)
-          tma_load_3d(q1_s + b * (BQ * 128), &p.tmQ1, qfull, b * 64, w.q0, w.bh);
+        for (int t = 0; t < NT; ++t) {
 #pragma unroll
-        for (int b = 0; b < D2 / 64; ++b)
-          tma_load_3d(q2_s + b * (BQ * 128), &p.tmQ2, qfull, b * 64, w.q0, w.bh);
+          for (int b = 0; b < D1 / 64; ++b)
+            tma_load_3d(q1_s(t) + b * (BQ * 128), &p.tmQ1, qfull, b * 64, w.q0 + t * BQ, w.bh);
+#pragma unroll
+          for (int b = 0; b < D2 / 64; ++b)
+            tma_load_3d(q2_s(t) + b * (BQ * 128), &p.tmQ2, qfull, b * 64, w.q0 + t * BQ, w.bh);
+        }
         armed_q = qph + 1;
         qph ^= 1;
-        for (int kt = 0; kt < w.nkt; ++kt) {
+        for (int kt = 0; kt < w.nkt_max; ++kt) {
           if (!(ok = mbar_wait(&kempty[ks], kph ^ 1, ctl))) break;
           mbar_arrive_expect_tx(&kfull[ks], Lay::stage_bytes);
 #pragma unroll
@@ -240,7 +275,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
           for (int b = 0; b < D2 / 64; ++b)
             tma_load_3d(k2_s(ks) + b * (BK * 128), &p.tmK2, &kfull[ks], b * 64, kt * BK, w.bh);
           armed_k[ks] = kph + 1;
-          if (++ks == KSTAGES) {
+          if (++ks == KS) {
             ks = 0;
             kph ^= 1;
           }
@@ -248,21 +283,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
       }
       if (!ok) {
         // Aborting: let the copies already in flight land before the CTA exits.
-        WaitCtl drainctl{abort_flag, p.status, p.wait_limit_ns};
         volatile int zero = 0;
-        drainctl.abort = &zero;
-        if (armed_q) mbar_wait(qfull, armed_q - 1, drainctl);
-        for (int s = 0; s < KSTAGES; ++s)
-          if (armed_k[s]) mbar_wait(&kfull[s], armed_k[s] - 1, drainctl);
+        WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
+        if (armed_q) mbar_wait(qfull, armed_q - 1, dctl);
+        for (int s = 0; s < KS; ++s)
+          if (armed_k[s]) mbar_wait(&kfull[s], armed_k[s] - 1, dctl);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(BQ, BK);
-      int ks = 0, sb = 0;
-      uint32_t kph = 0, sph = 0, qph = 0;
-      const uint32_t q1a = smem_u32(q1_s), q2a = smem_u32(q2_s);
+      int ks = 0;
+      int sb[NT] = {};
+      uint32_t kph = 0, qph = 0;
+      uint32_t sph[NT] = {};
       int u;
       bool ok = true;
       while (ok && sched.next(u)) {
@@ -270,47 +305,53 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
         if (!(ok = mbar_wait(qfull, qph, ctl))) break;
         qph ^= 1;
         tc_fence_after();
-        for (int kt = 0; kt < w.nkt; ++kt) {
+        for (int kt = 0; kt < w.nkt_max && ok; ++kt) {
           if (!(ok = mbar_wait(&kfull[ks], kph, ctl))) break;
-          if (!(ok = mbar_wait(&sempty[sb], sph ^ 1, ctl))) break;
-          tc_fence_after();
           const uint32_t k1a = smem_u32(k1_s(ks)), k2a = smem_u32(k2_s(ks));
-          const uint32_t t1 = tmem_base + sb * (2 * BK);
-          const uint32_t t2 = t1 + BK;
 #pragma unroll
-          for (int kk = 0; kk < D1 / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;
-            umma_bf16_ss(t1, sdesc_sw128(q1a + (kk >> 2) * (BQ * 128) + off, 16, 1024),
-                         sdesc_sw128(k1a + (kk >> 2) * (BK * 128) + off, 16, 1024), idesc, kk > 0);
-          }
+          for (int t = 0; t < NT; ++t) {
+            if (kt >= w.nkt[t]) continue;
+            if (!(ok = mbar_wait(&sempty[t * SBUF + sb[t]], sph[t] ^ 1, ctl))) break;
+            tc_fence_after();
+            const uint32_t q1a = smem_u32(q1_s(t)), q2a = smem_u32(q2_s(t));
+            const uint32_t t1 = tmem_base + (t * SBUF + sb[t]) * (2 * BK);
+            const uint32_t t2 = t1 + BK;
 #pragma unroll
-          for (int kk = 0; kk < D2 / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;
-            umma_bf16_ss(t2, sdesc_sw128(q2a + (kk >> 2) * (BQ * 128) + off, 16, 1024),
-                         sdesc_sw128(k2a + (kk >> 2) * (BK * 128) + off, 16, 1024), idesc, kk > 0);
+            for (int kk = 0; kk < D1 / 16; ++kk) {
+              const uint32_t o = (kk & 3) * 32;
+              umma_bf16_ss(t1, sdesc_sw128(q1a + (kk >> 2) * (BQ * 128) + o, 16, 1024),
+                           sdesc_sw128(k1a + (kk >> 2) * (BK * 128) + o, 16, 1024), idesc, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D2 / 16; ++kk) {
+              const uint32_t o = (kk & 3) * 32;
+              umma_bf16_ss(t2, sdesc_sw128(q2a + (kk >> 2) * (BQ * 128) + o, 16, 1024),
+                           sdesc_sw128(k2a + (kk >> 2) * (BK * 128) + o, 16, 1024), idesc, kk > 0);
+            }
+            umma_commit(&sfull[t * SBUF + sb[t]]);
+            if (++sb[t] == SBUF) {
+              sb[t] = 0;
+              sph[t] ^= 1;
+            }
           }
-          umma_commit(&sfull[sb]);
+          if (!ok) break;
           umma_commit(&kempty[ks]);
-          if (++ks == KSTAGES) {
+          if (++ks == KS) {
             ks = 0;
             kph ^= 1;
-          }
-          if (++sb == SBUF) {
-            sb = 0;
-            sph ^= 1;
           }
         }
         if (ok) umma_commit(qempty);
       }
       // Every UMMA issued by this thread completes before TMEM is released.
       umma_commit(drain);
-      WaitCtl drainctl{abort_flag, p.status, p.wait_limit_ns};
       volatile int zero = 0;
-      drainctl.abort = &zero;
-      mbar_wait(drain, 0, drainctl);
+      WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
+      mbar_wait(drain, 0, dctl);
     }
   } else {
     // ------------------------------------------------------------ reduction
+    const int t = (warp - 2) >> 2;  // query tile of this warpgroup
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t tlane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -321,14 +362,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     bool ok = true;
     while (ok && sched.next(u)) {
       const Unit w = decode_unit(p, u);
-      const int i_abs = w.q0 + row;
+      const int i_abs = w.q0 + t * BQ + row;
       const int lim = p.causal ? min(p.NK, i_abs + off + 1) : p.NK;  // visible keys [0, lim)
       RowState st{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
-      for (int kt = 0; kt < w.nkt; ++kt) {
-        if (!(ok = mbar_wait(&sfull[sb], sph, ctl))) break;
+      const int nkt = w.nkt[t];
+      for (int kt = 0; kt < nkt; ++kt) {
+        if (!(ok = mbar_wait(&sfull[t * SBUF + sb], sph, ctl))) break;
         tc_fence_after();
         uint32_t a[BK], b[BK];
-        const uint32_t tcol = tlane + sb * (2 * BK);
+        const uint32_t tcol = tlane + (t * SBUF + sb) * (2 * BK);
         tmem_ld_32x32b_x32(tcol + 0, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
         tmem_ld_32x32b_x32(tcol + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
         tmem_ld_32x32b_x32(tcol + BK, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
@@ -338,18 +380,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
         reg_fence(b);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sempty[sb]);
+        if (lane == 0) mbar_arrive(&sempty[t * SBUF + sb]);
         if (++sb == SBUF) {
           sb = 0;
           sph ^= 1;
         }
-        if (kt >= w.kt_mask)
+        if (kt >= w.kt_mask[t])
           tile_update<true>(a, b, p.c1, p.c2, lim - kt * BK, st);
         else
           tile_update<false>(a, b, p.c1, p.c2, BK, st);
       }
       if (!ok) break;
-      if (i_abs < p.NQ) {
+      if (nkt > 0 && i_abs < p.NQ) {
         const float lg1 = lg2(st.l1), lg2v = lg2(st.l2);
         const size_t o = static_cast<size_t>(w.bh) * p.NQ + i_abs;
         p.LSE1[o] = kLn2 * (st.m1 + lg1);
@@ -359,6 +401,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -9,8 +9,10 @@
 
 namespace skl {
 
-// Rows of Q in one forward tile (the UMMA M dimension and the TMEM lanes).
+// Rows of Q in one forward tile (the UMMA M dimension and the TMEM lanes);
+// a work unit holds kFwdTiles such tiles that share every key tile.
 constexpr int kFwdBQ = 128;
+constexpr int kFwdTiles = 2;
 // Keys per forward tile (UMMA N).
 constexpr int kFwdBK = 64;
 
@@ -34,12 +36,13 @@ cudaError_t launch_fwd(const FwdParams& p, int d1, int d2, int grid, cudaStream_
 // Keys per backward work unit (UMMA M of S^T and dK) and queries per step.
 constexpr int kBwdBK = 128;
 constexpr int kBwdBQ = 64;
-// Per-query-row record the backward reads: LSE1*log2e, LSE2*log2e, L, s1*dL, s2*dL, pad.
+// Per-query-row record the backward reads, stored field-major per 64-row step
+// ([step][field][64]): -LSE1*log2e, -LSE2*log2e, -L, s1*dL, s2*dL, 3 x pad.
 constexpr int kRowRec = 8;
 
 struct BwdParams {
   CUtensorMap tmQ1, tmK1, tmQ2, tmK2;  // Q maps: 64-row boxes; K maps: 128-row boxes
-  const float* rowrec;  // [BH][NQpad][kRowRec], NQpad = NQ rounded up to kBwdBQ
+  const float* rowrec;  // [BH][NQpad/64][kRowRec][64], NQpad = NQ rounded up to kBwdBQ
   float* dQacc;         // [BH][NQ][d1 + d2] fp32, zeroed before the main kernel
   __nv_bfloat16* dK1;   // [BH][NK][d1] or null
   __nv_bfloat16* dK2;   // [BH][NK][d2] or null
@@ -77,7 +80,9 @@ cudaError_t launch_bwd_convert(const BwdConvertParams& p, int num_sms, cudaStrea
 
 __host__ __device__ inline int bwd_units(int BH, int NK) { return BH * ((NK + kBwdBK - 1) / kBwdBK); }
 
-// Work units of the forward: (bh, 128-row query tile) pairs.
-__host__ __device__ inline int fwd_units(int BH, int NQ) { return BH * ((NQ + kFwdBQ - 1) / kFwdBQ); }
+// Work units of the forward: (bh, 256-row query block) pairs.
+__host__ __device__ inline int fwd_units(int BH, int NQ) {
+  return BH * ((NQ + kFwdBQ * kFwdTiles - 1) / (kFwdBQ * kFwdTiles));
+}
 
 }  // namespace skl

@@ -54,6 +54,10 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override H (smaller cases for profiling; not a bench line)")
+    ap.add_argument("--need", default="1111",
+                    help="which of dQ1 dK1 dQ2 dK2 the backward returns (e.g. 0101 = dK only)")
     return ap.parse_args(argv)
 
 
@@ -218,6 +222,8 @@ def run_reference(args, w: Workload, phase: str):
 def main(argv=None):
     args = parse_args(argv)
     w = WORKLOADS[args.workload]
+    if args.heads:
+        w = w.with_(H=args.heads)
     phase = args.phase if args.phase != "auto" else ("fwdbwd" if w.backward else "fwd")
     if args.impl == "reference":
         return run_reference(args, w, phase)
@@ -243,7 +249,8 @@ def main(argv=None):
     g = 1.0 / (w.B * w.H * w.NQ)
     dL = torch.full((w.B, w.H, w.NQ), g, device=dev)
     L, A, B = (torch.empty((w.B, w.H, w.NQ), device=dev) for _ in range(3))
-    grads = tuple(torch.empty_like(t) for t in (Q1, K1, Q2, K2))
+    need = tuple(c == "1" for c in args.need)
+    grads = tuple(torch.empty_like(t) if n else None for t, n in zip((Q1, K1, Q2, K2), need))
     ws = torch.empty(binding.workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal),
                      dtype=torch.uint8, device=dev)
 
@@ -368,7 +375,7 @@ def main(argv=None):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) teacher, student = teacher + noise; bf16)",
-        "config": {**workload_desc(w, phase),
+        "config": {**workload_desc(w, phase), **({"need": args.need} if args.need != "1111" else {}),
                    "parallelism": f"dp{world} (independent replicas, no collective)"},
         "pct_of_peak": value / world / peak,
         "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac_of_peak": fwd_tf / peak,
