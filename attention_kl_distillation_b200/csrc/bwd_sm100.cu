@@ -59,8 +59,14 @@ struct BwdLayout {
   static constexpr int rr_bytes = BQ * kRowRec * 4;
   static constexpr int qstage_bytes = q1_bytes + q2_bytes + rr_bytes;
   static constexpr int ds_bytes = BK * BQ * 2;  // one dS^T tile, bf16 [128 keys][64 queries]
-  static constexpr int QSTAGES = 2;
-  static constexpr int DSBUF = 2;
+  // Deepest Q ring (then most dS buffers) that fits: the Q tile of step t+2
+  // must be in flight while step t is contracted.
+  static constexpr int fixed_bytes = k1_bytes + k2_bytes + 1024 + 512;
+  static constexpr bool fits(int q, int d) {
+    return fixed_bytes + q * qstage_bytes + d * 2 * ds_bytes <= 232448;
+  }
+  static constexpr int QSTAGES = fits(4, 2) ? 4 : (fits(3, 2) ? 3 : (fits(4, 1) ? 4 : 3));
+  static constexpr int DSBUF = fits(QSTAGES, 2) ? 2 : 1;
   static constexpr int k1_off = 0;
   static constexpr int k2_off = k1_off + k1_bytes;
   static constexpr int q_off = k2_off + k2_bytes;
@@ -113,23 +119,20 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 
 // dS for one key row and HALF queries of a step (pairs of queries at a time,
 // packed f32x2).  s1/s2: raw products <K_t[key], Q_t[q]> from TMEM; rr: the
-// step's field-major row records offset to this half; writes the bf16 row
-// segments of s1*dS1^T and s2*dS2^T (HALF * 2 bytes each) into the swizzled
-// tiles at 16-byte chunks c0 .. c0 + HALF/8 - 1 of the key's 128-byte row.
+// step's field-major row records offset to this half; w1/w2 receive the bf16
+// pairs of s1*dS1^T and s2*dS2^T for these queries.
 //   u_t = log2 P_t = c_t S_t - LSE_t log2e
 //   dS1 = s1 dL P1 (ln2 (u1 - u2) - L),   dS2 = s2 dL (P2 - P1)
 // MASK: visible iff key < NK and (not causal or q >= thr), with thr the first
 // visible query index of this half for this key.
 template <bool MASK>
 __device__ __forceinline__ void form_ds(const uint32_t (&s1)[HALF], const uint32_t (&s2)[HALF],
-                                        const float* rr, float c1, float c2, int j, int c0,
-                                        bool key_ok, int thr, uint32_t ds1_row,
-                                        uint32_t ds2_row) {
+                                        const float* rr, float c1, float c2, bool key_ok, int thr,
+                                        uint32_t (&w1)[HALF / 2], uint32_t (&w2)[HALF / 2]) {
   const float2 C1 = make_float2(c1, c1), C2 = make_float2(c2, c2);
   const float2 NEG1 = make_float2(-1.f, -1.f), LN2 = make_float2(kLn2, kLn2);
 #pragma unroll
   for (int c = 0; c < HALF / 8; ++c) {
-    uint32_t w1[4], w2[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {  // 4 queries per h
       const int q = c * 8 + h * 4;
@@ -162,13 +165,23 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[HALF], const uint32
           d1.y = vy ? d1.y : 0.f;
           d2.y = vy ? d2.y : 0.f;
         }
-        w1[h * 2 + e] = pack_bf16(d1.x, d1.y);
-        w2[h * 2 + e] = pack_bf16(d2.x, d2.y);
+        w1[c * 4 + h * 2 + e] = pack_bf16(d1.x, d1.y);
+        w2[c * 4 + h * 2 + e] = pack_bf16(d2.x, d2.y);
       }
     }
+  }
+}
+
+// Stores the packed dS row segments of one key into the 128B-swizzled tiles:
+// 16-byte chunk c0 + c of row j lands at chunk (c0 + c) ^ (j mod 8).
+__device__ __forceinline__ void store_ds(const uint32_t (&w1)[HALF / 2],
+                                         const uint32_t (&w2)[HALF / 2], int j, int c0,
+                                         uint32_t ds1_row, uint32_t ds2_row) {
+#pragma unroll
+  for (int c = 0; c < HALF / 8; ++c) {
     const uint32_t sw = static_cast<uint32_t>(((c0 + c) ^ (j & 7)) << 4);
-    st_shared_v4(ds1_row + sw, w1[0], w1[1], w1[2], w1[3]);
-    st_shared_v4(ds2_row + sw, w2[0], w2[1], w2[2], w2[3]);
+    st_shared_v4(ds1_row + sw, w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
+    st_shared_v4(ds2_row + sw, w2[4 * c], w2[4 * c + 1], w2[4 * c + 2], w2[4 * c + 3]);
   }
 }
 
@@ -476,18 +489,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(sempty);
-        if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
-        dsph[db] ^= 1;
-        const uint32_t r1 = smem_u32(ds1_s(db)) + j * 128, r2 = smem_u32(ds2_s(db)) + j * 128;
         const float* rr = rr_s(qs) + half * HALF;
         const bool masked = (p.causal && q0 + off < w.k0 + BK - 1) || (w.k0 + BK > p.NK);
+        uint32_t w1[HALF / 2], w2[HALF / 2];
         if (masked) {
           // first visible query (index within this half) for this key
           const int thr = p.causal ? key - off - q0 - half * HALF : -1;
-          form_ds<true>(a, b, rr, p.c1, p.c2, j, half * (HALF / 8), key_ok, thr, r1, r2);
+          form_ds<true>(a, b, rr, p.c1, p.c2, key_ok, thr, w1, w2);
         } else {
-          form_ds<false>(a, b, rr, p.c1, p.c2, j, half * (HALF / 8), true, 0, r1, r2);
+          form_ds<false>(a, b, rr, p.c1, p.c2, true, 0, w1, w2);
         }
+        // the buffer is free once the contractions of the step that used it are done
+        if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
+        dsph[db] ^= 1;
+        store_ds(w1, w2, j, half * (HALF / 8), smem_u32(ds1_s(db)) + j * 128,
+                 smem_u32(ds2_s(db)) + j * 128);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&dsfull[db]);
