@@ -51,6 +51,10 @@ _lib.streamkl_query_device_status.restype = ctypes.c_int
 _lib.streamkl_set_wait_limit_ms.argtypes = [ctypes.c_int]
 _lib.streamkl_set_wait_limit_ms.restype = ctypes.c_int
 _lib.streamkl_abi_version.restype = ctypes.c_int
+_lib.streamkl_set_bwd_algorithm.argtypes = [ctypes.c_int]
+_lib.streamkl_set_bwd_algorithm.restype = ctypes.c_int
+_lib.streamkl_bwd_algorithm_for.argtypes = [_pp]
+_lib.streamkl_bwd_algorithm_for.restype = ctypes.c_int
 _lib.streamkl_launch_count.restype = ctypes.c_uint64
 
 
@@ -77,6 +81,22 @@ def status_string(st: int) -> str:
 def launch_count() -> int:
     """Kernels the library has launched in this process."""
     return int(_lib.streamkl_launch_count())
+
+
+BWD_ALGOS = {"auto": 0, "fused": 1, "split": 2}
+
+
+def set_bwd_algorithm(name: str) -> None:
+    """Process-wide backward algorithm: "auto", "fused" or "split"."""
+    st = _lib.streamkl_set_bwd_algorithm(BWD_ALGOS[name])
+    if st != OK:
+        raise StreamKLError(st, "streamkl_set_bwd_algorithm")
+
+
+def bwd_algorithm_for(B, H, NQ, NK, d1, d2, causal=False) -> str:
+    prob = problem(B, H, NQ, NK, d1, d2, causal)
+    code = _lib.streamkl_bwd_algorithm_for(ctypes.byref(prob))
+    return {v: k for k, v in BWD_ALGOS.items()}[code]
 
 
 def set_wait_limit_ms(ms: int) -> None:

@@ -20,15 +20,15 @@
 //                 dQ_t^T = K_t^T dS_t^T                     (M=d_t, N=64 queries)
 //               S for step t+1 is issued before the contractions of step t so
 //               that the tensor pipe works while dS is being formed.
-//   warps 2..9  two dS warpgroups, for queries 0..31 and 32..63 of a step:
+//   warps 2..17 four dS warpgroups, each for 16 of the 64 queries of a step:
 //               thread j owns key j (TMEM lane j), loads its S1^T and S2^T
 //               row segments, regenerates P1, P2 with exp2 on the MUFU pipe
 //               (packed f32x2 arithmetic elsewhere), forms s1*dS1 and s2*dS2
 //               in bf16 and writes them once to shared memory in the
 //               128B-swizzled layout that serves both as the K-major A operand
-//               of dK and the MN-major B operand of dQ^T.  Two warpgroups put
-//               two dS warps on every SM sub-partition.
-//   warps 10..13 dQ warpgroup: reads dQ^T (thread = feature index) and adds it
+//               of dK and the MN-major B operand of dQ^T.  Four warpgroups put
+//               four dS warps on every SM sub-partition to hide latencies.
+//   warps 18..21 dQ warpgroup: reads dQ^T (thread = feature index) and adds it
 //               into the fp32 workspace with coalesced reductions; at the end
 //               of a unit converts the dK accumulators to bf16 and stores them.
 // TMEM (512 columns): S1^T [0,64) S2^T [64,128) dK1 [128,128+d1) dK2 [..,+d2)
@@ -45,8 +45,11 @@ namespace {
 
 constexpr int BK = kBwdBK;  // keys per unit
 constexpr int BQ = kBwdBQ;  // queries per step
-constexpr int NTHREADS = 448;
-constexpr int HALF = BQ / 2;  // queries per dS warpgroup
+constexpr int kPrefetchSteps = 6;  // L2 prefetch distance of the producer, in steps
+constexpr int NDS = 4;          // dS warpgroups per CTA
+constexpr int QPW = BQ / NDS;   // queries of a step per dS warpgroup
+constexpr int DQ_WARP0 = 2 + 4 * NDS;
+constexpr int NTHREADS = (DQ_WARP0 + 4) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kColS1 = 0, kColS2 = 64, kColDK1 = 128, kColDQ1 = 384, kColDQ2 = 448;
 
@@ -85,7 +88,15 @@ struct BwdLayout {
 };
 
 struct UnitB {
-  int bh, k0, qt0, nsteps;
+  int bh, k0, qt0, nsteps, rot;
+  // Query tile of step t.  Steps start at a unit-dependent rotation: the sums
+  // over query tiles do not depend on the order, and rotating keeps the CTAs
+  // that work on one head from requesting the same Q tile at the same time.
+  __device__ __forceinline__ int qt(int t) const {
+    int r = t + rot;
+    if (r >= nsteps) r -= nsteps;
+    return qt0 + r;
+  }
 };
 
 __device__ __forceinline__ UnitB decode_unit(const BwdParams& p, int u) {
@@ -102,6 +113,7 @@ __device__ __forceinline__ UnitB decode_unit(const BwdParams& p, int u) {
   }
   w.qt0 = qt0;
   w.nsteps = nqt - qt0;
+  w.rot = static_cast<int>((static_cast<unsigned>(kt) * 2654435761u) % static_cast<unsigned>(w.nsteps));
   return w;
 }
 
@@ -117,7 +129,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-// dS for one key row and HALF queries of a step (pairs of queries at a time,
+// dS for one key row and QPW queries of a step (pairs of queries at a time,
 // packed f32x2).  s1/s2: raw products <K_t[key], Q_t[q]> from TMEM; rr: the
 // step's field-major row records offset to this half; w1/w2 receive the bf16
 // pairs of s1*dS1^T and s2*dS2^T for these queries.
@@ -126,13 +138,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // MASK: visible iff key < NK and (not causal or q >= thr), with thr the first
 // visible query index of this half for this key.
 template <bool MASK>
-__device__ __forceinline__ void form_ds(const uint32_t (&s1)[HALF], const uint32_t (&s2)[HALF],
+__device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_t (&s2)[QPW],
                                         const float* rr, float c1, float c2, bool key_ok, int thr,
-                                        uint32_t (&w1)[HALF / 2], uint32_t (&w2)[HALF / 2]) {
+                                        uint32_t (&w1)[QPW / 2], uint32_t (&w2)[QPW / 2]) {
   const float2 C1 = make_float2(c1, c1), C2 = make_float2(c2, c2);
   const float2 NEG1 = make_float2(-1.f, -1.f), LN2 = make_float2(kLn2, kLn2);
 #pragma unroll
-  for (int c = 0; c < HALF / 8; ++c) {
+  for (int c = 0; c < QPW / 8; ++c) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {  // 4 queries per h
       const int q = c * 8 + h * 4;
@@ -174,23 +186,23 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[HALF], const uint32
 
 // Stores the packed dS row segments of one key into the 128B-swizzled tiles:
 // 16-byte chunk c0 + c of row j lands at chunk (c0 + c) ^ (j mod 8).
-__device__ __forceinline__ void store_ds(const uint32_t (&w1)[HALF / 2],
-                                         const uint32_t (&w2)[HALF / 2], int j, int c0,
+__device__ __forceinline__ void store_ds(const uint32_t (&w1)[QPW / 2],
+                                         const uint32_t (&w2)[QPW / 2], int j, int c0,
                                          uint32_t ds1_row, uint32_t ds2_row) {
 #pragma unroll
-  for (int c = 0; c < HALF / 8; ++c) {
+  for (int c = 0; c < QPW / 8; ++c) {
     const uint32_t sw = static_cast<uint32_t>(((c0 + c) ^ (j & 7)) << 4);
     st_shared_v4(ds1_row + sw, w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
     st_shared_v4(ds2_row + sw, w2[4 * c], w2[4 * c + 1], w2[4 * c + 2], w2[4 * c + 3]);
   }
 }
 
-// Adds one dQ_t^T column block (64 queries of feature f) into the fp32
-// accumulator: base points at row q0, feature f; rows are LDQ floats apart.
+// Adds 32 queries of one dQ_t^T feature row into the fp32 accumulator: base
+// points at the first query's row, feature f; rows are LDQ floats apart.
 template <int LDQ, bool FULL>
-__device__ __forceinline__ void red_dq(float* base, const uint32_t (&v)[BQ], int nvalid) {
+__device__ __forceinline__ void red_dq(float* base, const uint32_t (&v)[32], int nvalid) {
 #pragma unroll
-  for (int i = 0; i < BQ; ++i)
+  for (int i = 0; i < 32; ++i)
     if (FULL || i < nvalid) atomicAdd(base + i * LDQ, __uint_as_float(v[i]));
 }
 
@@ -236,9 +248,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       mbar_init(&qempty[s], 1);
     }
     mbar_init(sfull, 1);
-    mbar_init(sempty, 8);  // every warp of both dS warpgroups
+    mbar_init(sempty, 4 * NDS);  // every warp of every dS warpgroup
     for (int s = 0; s < DSB; ++s) {
-      mbar_init(&dsfull[s], 8);
+      mbar_init(&dsfull[s], 4 * NDS);
       mbar_init(&dsempty[s], 1);
     }
     mbar_init(dqfull, 1);
@@ -248,7 +260,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
     mbar_init(dkempty, 4);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ufull[s], 1);
-      mbar_init(&uempty[s], 13);  // MMA thread + 8 dS warps + 4 dQ warps
+      mbar_init(&uempty[s], 1 + 4 * NDS + 4);  // MMA thread + dS warps + dQ warps
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -311,8 +323,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           tma_load_3d(k2_s + b * (BK * 128), &p.tmK2, kfull, b * 64, w.k0, w.bh);
         armed_k = kph + 1;
         kph ^= 1;
+        // Q tiles are re-read by every key tile of a head; a load that misses L2 takes
+        // longer than the ring hides, so each step also warms L2 a few steps ahead.
+        auto prefetch = [&](int t) {
+          if (t >= w.nsteps) return;
+          const int q0 = w.qt(t) * BQ;
+#pragma unroll
+          for (int b = 0; b < D1 / 64; ++b) tma_prefetch_l2_3d(&p.tmQ1, b * 64, q0, w.bh);
+#pragma unroll
+          for (int b = 0; b < D2 / 64; ++b) tma_prefetch_l2_3d(&p.tmQ2, b * 64, q0, w.bh);
+          bulk_prefetch_l2(p.rowrec + (static_cast<size_t>(w.bh) * p.NQpad + q0) * kRowRec,
+                           Lay::rr_bytes);
+        };
+        for (int t = 0; t < kPrefetchSteps; ++t) prefetch(t);
         for (int t = 0; t < w.nsteps; ++t) {
-          const int q0 = (w.qt0 + t) * BQ;
+          const int q0 = w.qt(t) * BQ;
+          prefetch(t + kPrefetchSteps);
           if (!(ok = mbar_wait(&qempty[qs], qph ^ 1, ctl))) break;
           mbar_arrive_expect_tx(&qfull[qs], Lay::qstage_bytes);
 #pragma unroll
@@ -451,9 +477,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
       mbar_wait(drain, 0, dctl);
     }
-  } else if (warp < 10) {
+  } else if (warp < DQ_WARP0) {
     // ------------------------------------------------------------ dS warpgroups
-    const int half = (warp - 2) >> 2;  // queries [half*32, half*32 + 32) of each step
+    const int part = (warp - 2) >> 2;  // queries [part*QPW, part*QPW + QPW) of each step
     const int quarter = warp & 3;
     const int j = quarter * 32 + lane;  // key row within the tile
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -475,26 +501,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       const int key = w.k0 + j;
       const bool key_ok = key < p.NK;
       for (int t = 0; t < w.nsteps; ++t) {
-        const int q0 = (w.qt0 + t) * BQ;
+        const int q0 = w.qt(t) * BQ;
         if (!(ok = mbar_wait(&qfull[qs], qph, ctl))) break;  // row records of this step
         if (!(ok = mbar_wait(sfull, sph, ctl))) break;
         sph ^= 1;
         tc_fence_after();
-        uint32_t a[HALF], b[HALF];
-        tmem_ld_32x32b_x32(tl + kColS1 + half * HALF, a);
-        tmem_ld_32x32b_x32(tl + kColS2 + half * HALF, b);
+        uint32_t a[QPW], b[QPW];
+        tmem_ld_32x32b_x16(tl + kColS1 + part * QPW, a);
+        tmem_ld_32x32b_x16(tl + kColS2 + part * QPW, b);
         tmem_ld_wait();
         reg_fence(a);
         reg_fence(b);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(sempty);
-        const float* rr = rr_s(qs) + half * HALF;
+        const float* rr = rr_s(qs) + part * QPW;
         const bool masked = (p.causal && q0 + off < w.k0 + BK - 1) || (w.k0 + BK > p.NK);
-        uint32_t w1[HALF / 2], w2[HALF / 2];
+        uint32_t w1[QPW / 2], w2[QPW / 2];
         if (masked) {
           // first visible query (index within this half) for this key
-          const int thr = p.causal ? key - off - q0 - half * HALF : -1;
+          const int thr = p.causal ? key - off - q0 - part * QPW : -1;
           form_ds<true>(a, b, rr, p.c1, p.c2, key_ok, thr, w1, w2);
         } else {
           form_ds<false>(a, b, rr, p.c1, p.c2, true, 0, w1, w2);
@@ -502,7 +528,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         // the buffer is free once the contractions of the step that used it are done
         if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
         dsph[db] ^= 1;
-        store_ds(w1, w2, j, half * (HALF / 8), smem_u32(ds1_s(db)) + j * 128,
+        store_ds(w1, w2, j, part * (QPW / 8), smem_u32(ds1_s(db)) + j * 128,
                  smem_u32(ds2_s(db)) + j * 128);
         fence_proxy_async_smem();
         __syncwarp();
@@ -538,7 +564,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       if (u < 0) break;
       const UnitB w = decode_unit(p, u);
       for (int t = 0; t < w.nsteps; ++t) {
-        const int q0 = (w.qt0 + t) * BQ;
+        const int q0 = w.qt(t) * BQ;
         if (!(ok = mbar_wait(dqfull, dqph, ctl))) break;
         dqph ^= 1;
         tc_fence_after();
@@ -549,22 +575,33 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           const bool want = tsel == 0 ? p.want_dq1 : p.want_dq2;
           const int f = tsel == 0 ? f1 : D1 + f2;
           const bool fok = (tsel == 0 ? f1 : f2) >= 0;
-          uint32_t v[BQ];
+          const uint32_t col = tl + (tsel == 0 ? kColDQ1 : kColDQ2);
+          // two halves of 32 queries; the slot is released once both are in registers
+          uint32_t v0[32], v1[32];
           if (want) {
-            const uint32_t col = tl + (tsel == 0 ? kColDQ1 : kColDQ2);
-            tmem_ld_32x32b_x32(col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-            tmem_ld_32x32b_x32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tmem_ld_32x32b_x32(col, v0);
             tmem_ld_wait();
-            reg_fence(v);
+            reg_fence(v0);
+          }
+          if (want && fok) {
+            if (nvalid == BQ)
+              red_dq<LDQ, true>(base + f, v0, 32);
+            else
+              red_dq<LDQ, false>(base + f, v0, nvalid);
+          }
+          if (want) {
+            tmem_ld_32x32b_x32(col + 32, v1);
+            tmem_ld_wait();
+            reg_fence(v1);
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&dqempty[tsel]);
           if (want && fok) {
             if (nvalid == BQ)
-              red_dq<LDQ, true>(base + f, v, BQ);
+              red_dq<LDQ, true>(base + 32 * LDQ + f, v1, 32);
             else
-              red_dq<LDQ, false>(base + f, v, nvalid);
+              red_dq<LDQ, false>(base + 32 * LDQ + f, v1, nvalid - 32);
           }
         }
       }
@@ -650,7 +687,11 @@ __global__ void streamkl_bwd_prep_kernel(const BwdPrepParams p) {
   const long long n4 = p.dqacc_elems / 4;
   for (long long e = tid; e < n4; e += stride)
     reinterpret_cast<float4*>(p.dQacc)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (tid == 0) *reinterpret_cast<int*>(p.rowrec + nrec * kRowRec) = 0;
+  if (tid == 0) {
+    int* counters = reinterpret_cast<int*>(p.rowrec + nrec * kRowRec);
+    counters[0] = 0;
+    counters[1] = 0;
+  }
 }
 
 // fp32 dQ accumulator [rows][d1 + d2] -> bf16 dQ1 [rows][d1], dQ2 [rows][d2].

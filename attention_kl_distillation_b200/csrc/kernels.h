@@ -73,6 +73,28 @@ struct BwdConvertParams {
   int d1, d2;
 };
 
+// Split backward (two passes of one kernel template): the dK pass streams
+// query tiles past resident 128-key tiles, the dQ pass streams key tiles past
+// resident 128-query tiles; each accumulates its gradient in TMEM and writes
+// it once, with no atomics and no dQ accumulator.
+enum class BwdPass : int { kDK = 0, kDQ = 1 };
+
+struct BwdSplitParams {
+  CUtensorMap tmR1, tmR2;  // resident operand maps (128-row boxes): K for dK, Q for dQ
+  CUtensorMap tmC1, tmC2;  // streamed operand maps (64-row boxes): Q for dK, K for dQ
+  const float* rowrec;     // [BH][NQpad/64][kRowRec][64]
+  int* counter;            // work-unit counter of this pass (zeroed by the prep kernel)
+  __nv_bfloat16* out1;     // dK1 or dQ1 (may be null)
+  __nv_bfloat16* out2;     // dK2 or dQ2 (may be null)
+  int BH, NQ, NK, NQpad, causal;
+  float c1, c2;
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+cudaError_t launch_bwd_split(const BwdSplitParams& p, BwdPass pass, int d1, int d2, int grid,
+                             cudaStream_t stream);
+
 size_t bwd_smem_bytes(int d1, int d2);
 cudaError_t launch_bwd(const BwdParams& p, int d1, int d2, int grid, cudaStream_t stream);
 cudaError_t launch_bwd_prep(const BwdPrepParams& p, int num_sms, cudaStream_t stream);

@@ -163,9 +163,39 @@ constexpr float kLog2e = 1.4426950408889634f;
 // records [BH][NQpad][8] fp32, then the work-unit counter; each part starts on
 // a 256-byte boundary.
 struct BwdWorkspace {
-  size_t dqacc_elems, rowrec_off, total;
+  size_t dqacc_elems, rowrec_off, counter_off, total;
   int NQpad;
 };
+
+// Backward algorithm: process-wide setting, environment default read once.
+int g_bwd_algo = -1;
+
+int bwd_algo_setting() {
+  if (g_bwd_algo < 0) {
+    int a = STREAMKL_BWD_AUTO;
+    if (const char* e = std::getenv("STREAMKL_BWD_ALGO")) {
+      if (!std::strcmp(e, "fused")) a = STREAMKL_BWD_FUSED;
+      else if (!std::strcmp(e, "split")) a = STREAMKL_BWD_SPLIT;
+    }
+    g_bwd_algo = a;
+  }
+  return g_bwd_algo;
+}
+
+// AUTO: the page keeps the fused kernel while its dQ reductions stay cheap and
+// switches to separate kernels when they contend.  On B200 the fused kernel
+// measured faster up to the largest accumulator tested (B1 H32 N16384 d128:
+// 537 MB of fp32 dQ, fused 9.9 ms vs split 10.7 ms), so the threshold sits
+// above every measured shape; set the algorithm explicitly to override.
+constexpr size_t kFusedDqAccLimit = 4ull << 30;
+
+streamkl_bwd_algorithm resolve_bwd_algo(const streamkl_problem& pr) {
+  const int a = bwd_algo_setting();
+  if (a == STREAMKL_BWD_FUSED || a == STREAMKL_BWD_SPLIT) return static_cast<streamkl_bwd_algorithm>(a);
+  const size_t acc = static_cast<size_t>(pr.B) * pr.H * static_cast<size_t>(pr.NQ) *
+                     static_cast<size_t>(pr.d1 + pr.d2) * sizeof(float);
+  return acc > kFusedDqAccLimit ? STREAMKL_BWD_SPLIT : STREAMKL_BWD_FUSED;
+}
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -176,7 +206,8 @@ BwdWorkspace bwd_workspace_layout(const streamkl_problem& pr) {
   w.dqacc_elems = BH * static_cast<size_t>(pr.NQ) * static_cast<size_t>(pr.d1 + pr.d2);
   w.rowrec_off = round256(w.dqacc_elems * sizeof(float));
   const size_t rec = BH * static_cast<size_t>(w.NQpad) * skl::kRowRec * sizeof(float);
-  w.total = w.rowrec_off + round256(rec + sizeof(int));
+  w.counter_off = w.rowrec_off + rec;  // two work-unit counters follow the records
+  w.total = w.rowrec_off + round256(rec + 2 * sizeof(int));
   return w;
 }
 
@@ -198,6 +229,18 @@ const char* streamkl_status_string(streamkl_status st) {
     case STREAMKL_EDEVICE: return "device-side error";
   }
   return "unknown status";
+}
+
+streamkl_status streamkl_set_bwd_algorithm(streamkl_bwd_algorithm algo) {
+  if (algo != STREAMKL_BWD_AUTO && algo != STREAMKL_BWD_FUSED && algo != STREAMKL_BWD_SPLIT)
+    return STREAMKL_EINVAL;
+  g_bwd_algo = algo;
+  return STREAMKL_OK;
+}
+
+streamkl_bwd_algorithm streamkl_bwd_algorithm_for(const streamkl_problem* prob) {
+  if (check_problem(prob) != STREAMKL_OK) return STREAMKL_BWD_AUTO;
+  return resolve_bwd_algo(*prob);
 }
 
 streamkl_status streamkl_set_wait_limit_ms(int ms) {
@@ -305,7 +348,8 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   float* rowrec = reinterpret_cast<float*>(ws + lay.rowrec_off);
   const float s1 = scale_or_default(prob->s1, prob->d1);
   const float s2 = scale_or_default(prob->s2, prob->d2);
-  const bool want_dq = dQ1 || dQ2;
+  const bool split = resolve_bwd_algo(*prob) == STREAMKL_BWD_SPLIT;
+  const bool want_dq = (dQ1 || dQ2) && !split;  // the fused path accumulates dQ in fp32
 
   skl::BwdPrepParams pp;
   pp.L = L;
@@ -322,6 +366,50 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   pp.s2 = s2;
   if (skl::launch_bwd_prep(pp, dev->num_sms, s) != cudaSuccess) return STREAMKL_ECUDA;
   g_launches.fetch_add(1);
+
+  if (split) {
+    int* counters = reinterpret_cast<int*>(ws + lay.counter_off);
+    skl::BwdSplitParams sp;
+    sp.rowrec = rowrec;
+    sp.BH = static_cast<int>(BH);
+    sp.NQ = prob->NQ;
+    sp.NK = prob->NK;
+    sp.NQpad = lay.NQpad;
+    sp.causal = prob->causal;
+    sp.c1 = s1 * kLog2e;
+    sp.c2 = s2 * kLog2e;
+    sp.status = dev->status;
+    sp.wait_limit_ns = wait_limit_ns();
+    if (dK1 || dK2) {  // dK pass: resident key tiles, streamed query tiles
+      if ((st = tensor_map(K1, BH, prob->NK, prob->d1, 128, &sp.tmR1)) != STREAMKL_OK) return st;
+      if ((st = tensor_map(K2, BH, prob->NK, prob->d2, 128, &sp.tmR2)) != STREAMKL_OK) return st;
+      if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, 64, &sp.tmC1)) != STREAMKL_OK) return st;
+      if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, 64, &sp.tmC2)) != STREAMKL_OK) return st;
+      sp.counter = counters;
+      sp.out1 = static_cast<__nv_bfloat16*>(dK1);
+      sp.out2 = static_cast<__nv_bfloat16*>(dK2);
+      const int units = static_cast<int>(BH) * ((prob->NK + 127) / 128);
+      if (skl::launch_bwd_split(sp, skl::BwdPass::kDK, prob->d1, prob->d2,
+                                units < dev->num_sms ? units : dev->num_sms, s) != cudaSuccess)
+        return STREAMKL_ECUDA;
+      g_launches.fetch_add(1);
+    }
+    if (dQ1 || dQ2) {  // dQ pass: resident query tiles, streamed key tiles
+      if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, 128, &sp.tmR1)) != STREAMKL_OK) return st;
+      if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, 128, &sp.tmR2)) != STREAMKL_OK) return st;
+      if ((st = tensor_map(K1, BH, prob->NK, prob->d1, 64, &sp.tmC1)) != STREAMKL_OK) return st;
+      if ((st = tensor_map(K2, BH, prob->NK, prob->d2, 64, &sp.tmC2)) != STREAMKL_OK) return st;
+      sp.counter = counters + 1;
+      sp.out1 = static_cast<__nv_bfloat16*>(dQ1);
+      sp.out2 = static_cast<__nv_bfloat16*>(dQ2);
+      const int units = static_cast<int>(BH) * ((prob->NQ + 127) / 128);
+      if (skl::launch_bwd_split(sp, skl::BwdPass::kDQ, prob->d1, prob->d2,
+                                units < dev->num_sms ? units : dev->num_sms, s) != cudaSuccess)
+        return STREAMKL_ECUDA;
+      g_launches.fetch_add(1);
+    }
+    return STREAMKL_OK;
+  }
 
   skl::BwdParams p;
   if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, skl::kBwdBQ, &p.tmQ1)) != STREAMKL_OK) return st;

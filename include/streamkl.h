@@ -135,6 +135,33 @@ streamkl_status streamkl_bwd_noalloc(const streamkl_problem *prob, const float *
                                      const float *LSE2, void *dQ1, void *dK1, void *dQ2,
                                      void *dK2, streamkl_stream_t stream);
 
+/*
+ * How streamkl_bwd computes the gradients (section 2, "Fusione del Kernel",
+ * and the fused-versus-separate ablation):
+ *  FUSED  one kernel visits every (query tile, key tile) pair once; dK stays
+ *         on chip, dQ is accumulated across key tiles with fp32 reductions
+ *         into the workspace, then converted to bf16.
+ *  SPLIT  two passes of one kernel: a dK pass over key tiles and a dQ pass
+ *         over query tiles, each regenerating the probabilities; no
+ *         reductions in global memory.
+ *  AUTO   FUSED unless the fp32 dQ accumulator (B*H*NQ*(d1+d2)*4 bytes)
+ *         exceeds 4 GiB; on B200 the fused kernel measured faster at every
+ *         size tested.
+ * Results agree within rounding either way.  Process-wide; default AUTO (or
+ * the environment variable STREAMKL_BWD_ALGO = auto | fused | split, read
+ * once).
+ */
+typedef enum {
+  STREAMKL_BWD_AUTO = 0,
+  STREAMKL_BWD_FUSED = 1,
+  STREAMKL_BWD_SPLIT = 2
+} streamkl_bwd_algorithm;
+
+streamkl_status streamkl_set_bwd_algorithm(streamkl_bwd_algorithm algo);
+
+/* The algorithm streamkl_bwd would use for this problem (AUTO resolved). */
+streamkl_bwd_algorithm streamkl_bwd_algorithm_for(const streamkl_problem *prob);
+
 /* Static English text for a status code. */
 const char *streamkl_status_string(streamkl_status st);
 

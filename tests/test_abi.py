@@ -106,3 +106,20 @@ def test_binding_argtypes_match_header():
         fn = getattr(B.lib(), name)
         if fn.argtypes is not None:
             assert len(fn.argtypes) == len(params), name
+
+
+def test_bwd_algorithm_selection():
+    lib = B.lib()
+    assert lib.streamkl_set_bwd_algorithm(7) == B.EINVAL
+    try:
+        B.set_bwd_algorithm("fused")
+        assert B.bwd_algorithm_for(1, 32, 16384, 16384, 128, 128, True) == "fused"
+        B.set_bwd_algorithm("split")
+        assert B.bwd_algorithm_for(1, 2, 256, 256, 64, 64) == "split"
+        B.set_bwd_algorithm("auto")
+        # AUTO: fused unless the fp32 dQ accumulator exceeds 4 GiB
+        assert B.bwd_algorithm_for(1, 2, 256, 256, 64, 64) == "fused"
+        assert B.bwd_algorithm_for(1, 32, 16384, 16384, 128, 128, True) == "fused"
+        assert B.bwd_algorithm_for(4, 32, 65536, 65536, 128, 128, True) == "split"
+    finally:
+        B.set_bwd_algorithm("auto")

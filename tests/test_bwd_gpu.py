@@ -7,6 +7,15 @@ from gpu_common import TOL_GRAD, cuda_inputs, oracle_bits, rel_frobenius, worklo
 
 pytestmark = pytest.mark.gpu
 
+
+@pytest.fixture(autouse=True, params=["fused", "split"])
+def bwd_algo(request):
+    """Every backward test runs with both algorithms of streamkl_bwd."""
+    from attention_kl_distillation_b200 import set_bwd_algorithm
+    set_bwd_algorithm(request.param)
+    yield request.param
+    set_bwd_algorithm("auto")
+
 SHAPES = [  # B, H, NQ, NK, d1, d2, causal
     (1, 1, 64, 128, 64, 64, False),
     (1, 2, 130, 200, 128, 128, True),
