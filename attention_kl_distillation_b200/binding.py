@@ -51,6 +51,8 @@ _lib.streamkl_query_device_status.restype = ctypes.c_int
 _lib.streamkl_set_wait_limit_ms.argtypes = [ctypes.c_int]
 _lib.streamkl_set_wait_limit_ms.restype = ctypes.c_int
 _lib.streamkl_abi_version.restype = ctypes.c_int
+_lib.streamkl_debug_inject.argtypes = [ctypes.c_int]
+_lib.streamkl_debug_inject.restype = ctypes.c_int
 _lib.streamkl_set_bwd_algorithm.argtypes = [ctypes.c_int]
 _lib.streamkl_set_bwd_algorithm.restype = ctypes.c_int
 _lib.streamkl_bwd_algorithm_for.argtypes = [_pp]
@@ -97,6 +99,13 @@ def bwd_algorithm_for(B, H, NQ, NK, d1, d2, causal=False) -> str:
     prob = problem(B, H, NQ, NK, d1, d2, causal)
     code = _lib.streamkl_bwd_algorithm_for(ctypes.byref(prob))
     return {v: k for k, v in BWD_ALGOS.items()}[code]
+
+
+def debug_inject(mode: int) -> None:
+    """Arm (1) or disarm (0) the one-shot stalled-producer fault of the next forward."""
+    st = _lib.streamkl_debug_inject(int(mode))
+    if st != OK:
+        raise StreamKLError(st, "streamkl_debug_inject")
 
 
 def set_wait_limit_ms(ms: int) -> None:

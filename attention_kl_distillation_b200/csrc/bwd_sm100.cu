@@ -20,15 +20,15 @@
 //                 dQ_t^T = K_t^T dS_t^T                     (M=d_t, N=64 queries)
 //               S for step t+1 is issued before the contractions of step t so
 //               that the tensor pipe works while dS is being formed.
-//   warps 2..17 four dS warpgroups, each for 16 of the 64 queries of a step:
+//   warps 2..9  two dS warpgroups, each for 32 of the 64 queries of a step:
 //               thread j owns key j (TMEM lane j), loads its S1^T and S2^T
 //               row segments, regenerates P1, P2 with exp2 on the MUFU pipe
 //               (packed f32x2 arithmetic elsewhere), forms s1*dS1 and s2*dS2
 //               in bf16 and writes them once to shared memory in the
 //               128B-swizzled layout that serves both as the K-major A operand
-//               of dK and the MN-major B operand of dQ^T.  Four warpgroups put
-//               four dS warps on every SM sub-partition to hide latencies.
-//   warps 18..21 dQ warpgroup: reads dQ^T (thread = feature index) and adds it
+//               of dK and the MN-major B operand of dQ^T.  Two warpgroups put
+//               two dS warps on every SM sub-partition.
+//   warps 10..13 dQ warpgroup: reads dQ^T (thread = feature index) and adds it
 //               into the fp32 workspace with coalesced reductions; at the end
 //               of a unit converts the dK accumulators to bf16 and stores them.
 // TMEM (512 columns): S1^T [0,64) S2^T [64,128) dK1 [128,128+d1) dK2 [..,+d2)
@@ -45,8 +45,7 @@ namespace {
 
 constexpr int BK = kBwdBK;  // keys per unit
 constexpr int BQ = kBwdBQ;  // queries per step
-constexpr int kPrefetchSteps = 6;  // L2 prefetch distance of the producer, in steps
-constexpr int NDS = 4;          // dS warpgroups per CTA
+constexpr int NDS = 2;          // dS warpgroups per CTA
 constexpr int QPW = BQ / NDS;   // queries of a step per dS warpgroup
 constexpr int DQ_WARP0 = 2 + 4 * NDS;
 constexpr int NTHREADS = (DQ_WARP0 + 4) * 32;
@@ -89,9 +88,8 @@ struct BwdLayout {
 
 struct UnitB {
   int bh, k0, qt0, nsteps, rot;
-  // Query tile of step t.  Steps start at a unit-dependent rotation: the sums
-  // over query tiles do not depend on the order, and rotating keeps the CTAs
-  // that work on one head from requesting the same Q tile at the same time.
+  // Query tile of step t (steps may start at a rotation rot; the sums over
+  // query tiles do not depend on the order).
   __device__ __forceinline__ int qt(int t) const {
     int r = t + rot;
     if (r >= nsteps) r -= nsteps;
@@ -113,7 +111,7 @@ __device__ __forceinline__ UnitB decode_unit(const BwdParams& p, int u) {
   }
   w.qt0 = qt0;
   w.nsteps = nqt - qt0;
-  w.rot = static_cast<int>((static_cast<unsigned>(kt) * 2654435761u) % static_cast<unsigned>(w.nsteps));
+  w.rot = 0;
   return w;
 }
 
@@ -323,22 +321,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           tma_load_3d(k2_s + b * (BK * 128), &p.tmK2, kfull, b * 64, w.k0, w.bh);
         armed_k = kph + 1;
         kph ^= 1;
-        // Q tiles are re-read by every key tile of a head; a load that misses L2 takes
-        // longer than the ring hides, so each step also warms L2 a few steps ahead.
-        auto prefetch = [&](int t) {
-          if (t >= w.nsteps) return;
-          const int q0 = w.qt(t) * BQ;
-#pragma unroll
-          for (int b = 0; b < D1 / 64; ++b) tma_prefetch_l2_3d(&p.tmQ1, b * 64, q0, w.bh);
-#pragma unroll
-          for (int b = 0; b < D2 / 64; ++b) tma_prefetch_l2_3d(&p.tmQ2, b * 64, q0, w.bh);
-          bulk_prefetch_l2(p.rowrec + (static_cast<size_t>(w.bh) * p.NQpad + q0) * kRowRec,
-                           Lay::rr_bytes);
-        };
-        for (int t = 0; t < kPrefetchSteps; ++t) prefetch(t);
         for (int t = 0; t < w.nsteps; ++t) {
           const int q0 = w.qt(t) * BQ;
-          prefetch(t + kPrefetchSteps);
           if (!(ok = mbar_wait(&qempty[qs], qph ^ 1, ctl))) break;
           mbar_arrive_expect_tx(&qfull[qs], Lay::qstage_bytes);
 #pragma unroll
@@ -507,8 +491,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         sph ^= 1;
         tc_fence_after();
         uint32_t a[QPW], b[QPW];
-        tmem_ld_32x32b_x16(tl + kColS1 + part * QPW, a);
-        tmem_ld_32x32b_x16(tl + kColS2 + part * QPW, b);
+        tmem_ld_32x32b<QPW>(tl + kColS1 + part * QPW, a);
+        tmem_ld_32x32b<QPW>(tl + kColS2 + part * QPW, b);
         tmem_ld_wait();
         reg_fence(a);
         reg_fence(b);

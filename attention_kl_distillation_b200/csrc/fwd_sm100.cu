@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
         }
         armed_q = qph + 1;
         qph ^= 1;
-        for (int kt = 0; kt < w.nkt_max; ++kt) {
+        for (int kt = 0; kt < (p.withhold_keys ? 0 : w.nkt_max); ++kt) {
           if (!(ok = mbar_wait(&kempty[ks], kph ^ 1, ctl))) break;
           mbar_arrive_expect_tx(&kfull[ks], Lay::stage_bytes);
 #pragma unroll

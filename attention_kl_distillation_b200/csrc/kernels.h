@@ -25,6 +25,7 @@ struct FwdParams {
   float c1, c2;  // s_t * log2(e): logits in the base-2 domain
   int* status;   // device status word
   unsigned long long wait_limit_ns;
+  int withhold_keys;  // test hook: the producer issues no key tiles (waits then time out)
 };
 
 // Dynamic shared memory the forward kernel needs for head dims (d1, d2).

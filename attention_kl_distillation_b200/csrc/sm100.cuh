@@ -256,6 +256,17 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       : "memory");
 }
 
+// 32 lanes x N consecutive 32-bit columns, N = 16 or 32.
+template <int N>
+__device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N == 16 || N == 32, "16 or 32 columns");
+  if constexpr (N == 32) {
+    tmem_ld_32x32b_x32(taddr, r);
+  } else {
+    tmem_ld_32x32b_x16(taddr, r);
+  }
+}
+
 // 32 lanes x 8 consecutive 32-bit columns, registers -> TMEM.
 __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile(

@@ -25,6 +25,7 @@ __device__ int g_device_status;  // set by kernels (atomicCAS from 0), read + cl
 constexpr int kMaxDevices = 64;
 
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_fault_mode{0};  // one-shot test hook, see streamkl_debug_inject
 
 struct DeviceInfo {
   bool probed = false;
@@ -231,6 +232,12 @@ const char* streamkl_status_string(streamkl_status st) {
   return "unknown status";
 }
 
+streamkl_status streamkl_debug_inject(int mode) {
+  if (mode != 0 && mode != 1) return STREAMKL_EINVAL;
+  g_fault_mode.store(mode);
+  return STREAMKL_OK;
+}
+
 streamkl_status streamkl_set_bwd_algorithm(streamkl_bwd_algorithm algo) {
   if (algo != STREAMKL_BWD_AUTO && algo != STREAMKL_BWD_FUSED && algo != STREAMKL_BWD_SPLIT)
     return STREAMKL_EINVAL;
@@ -300,6 +307,7 @@ streamkl_status streamkl_fwd(const streamkl_problem* prob, const void* Q1, const
   p.c2 = scale_or_default(prob->s2, prob->d2) * kLog2e;
   p.status = dev->status;
   p.wait_limit_ns = wait_limit_ns();
+  p.withhold_keys = g_fault_mode.exchange(0) == 1 ? 1 : 0;
   const int units = skl::fwd_units(p.BH, p.NQ);
   const int grid = units < dev->num_sms ? units : dev->num_sms;
   if (skl::launch_fwd(p, prob->d1, prob->d2, grid, reinterpret_cast<cudaStream_t>(stream)) !=

@@ -242,6 +242,7 @@ def main(argv=None):
 
     import attention_kl_distillation_b200 as skl
     from attention_kl_distillation_b200 import binding
+    from attention_kl_distillation_b200.parallel import max_over_ranks
 
     dev = torch.device("cuda", local)
     cpu_ins = make_inputs(w, seed=w.seed + rank)  # independent replica per rank
@@ -296,11 +297,7 @@ def main(argv=None):
     if skl.query_device_status() != 0:
         raise RuntimeError("device status reported an error in the timed region")
 
-    total_ms = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), device=dev)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) if phase == "fwdbwd" else 0.0
     fl_step = step_flops(w, phase)
@@ -353,11 +350,7 @@ def main(argv=None):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
         e2e = {"value": world * fl_step * ke / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / ke, "api": "attention_kl_distillation_b200.streamkl"}

@@ -179,6 +179,16 @@ streamkl_status streamkl_query_device_status(streamkl_stream_t stream);
  */
 streamkl_status streamkl_set_wait_limit_ms(int ms);
 
+/*
+ * Test hook for failure detection (no counterpart on the page).  mode 1 arms a
+ * one-shot fault: in the next streamkl_fwd launch the TMA producer issues no
+ * key tiles, so the UMMA warp's wait for them runs past the wait limit.  The
+ * kernel then records STREAMKL_ETIMEOUT, every role of every CTA unwinds (in-
+ * flight copies land, TMEM is freed) and the launch ends; the CUDA context
+ * stays usable.  mode 0 disarms.  Nothing faults, traps or hangs.
+ */
+streamkl_status streamkl_debug_inject(int mode);
+
 /* Version of this ABI: 1. */
 int streamkl_abi_version(void);
 
