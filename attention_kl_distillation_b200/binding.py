@@ -38,6 +38,12 @@ _vp = ctypes.c_void_p
 _pp = ctypes.POINTER(Problem)
 _lib.streamkl_fwd.argtypes = [_pp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.streamkl_fwd.restype = ctypes.c_int
+_lib.streamkl_fwd_splitk.argtypes = [_pp] + [_vp] * 7 + [ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+_lib.streamkl_fwd_splitk.restype = ctypes.c_int
+_lib.streamkl_fwd_splitk_workspace_size.argtypes = [_pp, ctypes.c_int]
+_lib.streamkl_fwd_splitk_workspace_size.restype = ctypes.c_size_t
+_lib.streamkl_fwd_splitk_suggest.argtypes = [_pp]
+_lib.streamkl_fwd_splitk_suggest.restype = ctypes.c_int
 _lib.streamkl_bwd_workspace_size.argtypes = [_pp]
 _lib.streamkl_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.streamkl_bwd.argtypes = [_pp] + [_vp] * 13 + [ctypes.c_size_t, _vp]
@@ -159,6 +165,38 @@ def fwd(Q1, K1, Q2, K2, causal=False, s1=None, s2=None, out=None):
                                _ptr(L), _ptr(A), _ptr(Bv), _stream(Q1.device))
     if st != OK:
         raise StreamKLError(st, "streamkl_fwd")
+    return L, A, Bv
+
+
+def splitk_workspace_size(B, H, NQ, NK, d1, d2, nsplit, causal=False) -> int:
+    prob = problem(B, H, NQ, NK, d1, d2, causal)
+    return int(_lib.streamkl_fwd_splitk_workspace_size(ctypes.byref(prob), int(nsplit)))
+
+
+def fwd_splitk(Q1, K1, Q2, K2, causal=False, s1=None, s2=None, nsplit=None, workspace=None,
+               out=None):
+    """streamkl_fwd_splitk: the forward with the keys split across CTAs (small N_Q).
+    nsplit=None asks the library for a split that fills the device."""
+    B, H, NQ, NK, d1, d2 = _check_qk(Q1, K1, Q2, K2)
+    prob = problem(B, H, NQ, NK, d1, d2, causal, s1, s2)
+    with torch.cuda.device(Q1.device):
+        if nsplit is None:
+            nsplit = int(_lib.streamkl_fwd_splitk_suggest(ctypes.byref(prob)))
+            if nsplit < 1:
+                raise StreamKLError(EINVAL, "streamkl_fwd_splitk_suggest")
+        need = int(_lib.streamkl_fwd_splitk_workspace_size(ctypes.byref(prob), int(nsplit)))
+        if workspace is None:
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=Q1.device)
+        if out is None:
+            out = tuple(torch.empty((B, H, NQ), dtype=torch.float32, device=Q1.device)
+                        for _ in range(3))
+        L, A, Bv = out
+        st = _lib.streamkl_fwd_splitk(ctypes.byref(prob), _ptr(Q1), _ptr(K1), _ptr(Q2), _ptr(K2),
+                                      _ptr(L), _ptr(A), _ptr(Bv), int(nsplit), _ptr(workspace),
+                                      ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                      _stream(Q1.device))
+    if st != OK:
+        raise StreamKLError(st, "streamkl_fwd_splitk")
     return L, A, Bv
 
 

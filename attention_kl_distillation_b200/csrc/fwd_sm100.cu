@@ -85,29 +85,38 @@ struct Sched {
 
 struct Unit {
   int bh, q0;
-  int nkt[NT];     // key tiles each query tile needs (0: tile holds no valid row)
+  int kt_lo;       // first key tile of this unit (split-K chunk start; 0 without split)
+  int nkt[NT];     // end of the key tiles each query tile processes (<= kt_lo: none)
   int kt_mask[NT]; // key tiles [kt_mask, nkt) need element masks
   int nkt_max;
+  int split;       // key split index (0 without split)
 };
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   const int nqb = (p.NQ + BQ * NT - 1) / (BQ * NT);
   Unit w;
+  w.split = 0;
+  if (p.nsplit > 1) {
+    w.split = u % p.nsplit;
+    u /= p.nsplit;
+  }
   w.bh = u % p.BH;
   w.q0 = (nqb - 1 - u / p.BH) * (BQ * NT);  // longest (last) query blocks first
   const int nkt_all = (p.NK + BK - 1) / BK;
   const int tail = (p.NK % BK) ? nkt_all - 1 : nkt_all;
   const int off = p.NK - p.NQ;
-  w.nkt_max = 0;
+  w.kt_lo = p.nsplit > 1 ? w.split * p.kt_chunk : 0;
+  const int kt_hi = p.nsplit > 1 ? min(nkt_all, w.kt_lo + p.kt_chunk) : nkt_all;
+  w.nkt_max = w.kt_lo;
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
     const int r0 = w.q0 + t * BQ;
-    int nkt = nkt_all, km = tail;
+    int nkt = kt_hi, km = tail;
     if (r0 >= p.NQ) {
       nkt = 0;
     } else if (p.causal) {
       const int last = min(r0 + BQ - 1, p.NQ - 1) + off;  // last key any row of the tile sees
-      nkt = min(nkt_all, last / BK + 1);
+      nkt = min(kt_hi, last / BK + 1);
       km = min(km, (r0 + off + 1) / BK);  // first tile the first row cannot fully see
     }
     w.nkt[t] = nkt;
@@ -236,7 +245,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  Sched sched{fwd_units(p.BH, p.NQ), static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x), 0};
+  Sched sched{fwd_units(p.BH, p.NQ, p.nsplit), static_cast<int>(gridDim.x),
+              static_cast<int>(blockIdx.x), 0};
   auto q1_s = [&](int t) { return smem + Lay::q1_off + t * Lay::q1_tile; };
   auto q2_s = [&](int t) { return smem + Lay::q2_off + t * Lay::q2_tile; };
   auto k1_s = [&](int s) { return smem + Lay::k_off + s * Lay::stage_bytes; };
@@ -252,6 +262,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
       bool ok = true;
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
+        if (w.nkt_max <= w.kt_lo) continue;  // split chunk past every row's frontier
         if (!(ok = mbar_wait(qempty, qph ^ 1, ctl))) break;
         mbar_arrive_expect_tx(qfull, Lay::q_bytes);
 #pragma unroll
@@ -265,7 +276,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
         }
         armed_q = qph + 1;
         qph ^= 1;
-        for (int kt = 0; kt < (p.withhold_keys ? 0 : w.nkt_max); ++kt) {
+        for (int kt = w.kt_lo; kt < (p.withhold_keys ? w.kt_lo : w.nkt_max); ++kt) {
           if (!(ok = mbar_wait(&kempty[ks], kph ^ 1, ctl))) break;
           mbar_arrive_expect_tx(&kfull[ks], Lay::stage_bytes);
 #pragma unroll
@@ -302,10 +313,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
       bool ok = true;
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
+        if (w.nkt_max <= w.kt_lo) continue;
         if (!(ok = mbar_wait(qfull, qph, ctl))) break;
         qph ^= 1;
         tc_fence_after();
-        for (int kt = 0; kt < w.nkt_max && ok; ++kt) {
+        for (int kt = w.kt_lo; kt < w.nkt_max && ok; ++kt) {
           if (!(ok = mbar_wait(&kfull[ks], kph, ctl))) break;
           const uint32_t k1a = smem_u32(k1_s(ks)), k2a = smem_u32(k2_s(ks));
 #pragma unroll
@@ -362,11 +374,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     bool ok = true;
     while (ok && sched.next(u)) {
       const Unit w = decode_unit(p, u);
+      if (w.nkt_max <= w.kt_lo) continue;
       const int i_abs = w.q0 + t * BQ + row;
       const int lim = p.causal ? min(p.NK, i_abs + off + 1) : p.NK;  // visible keys [0, lim)
       RowState st{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
       const int nkt = w.nkt[t];
-      for (int kt = 0; kt < nkt; ++kt) {
+      for (int kt = w.kt_lo; kt < nkt; ++kt) {
         if (!(ok = mbar_wait(&sfull[t * SBUF + sb], sph, ctl))) break;
         tc_fence_after();
         uint32_t a[BK], b[BK];
@@ -391,12 +404,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
           tile_update<false>(a, b, p.c1, p.c2, BK, st);
       }
       if (!ok) break;
-      if (nkt > 0 && i_abs < p.NQ) {
-        const float lg1 = lg2(st.l1), lg2v = lg2(st.l2);
+      if (i_abs < p.NQ && w.q0 + t * BQ < p.NQ) {
         const size_t o = static_cast<size_t>(w.bh) * p.NQ + i_abs;
-        p.LSE1[o] = kLn2 * (st.m1 + lg1);
-        p.LSE2[o] = kLn2 * (st.m2 + lg2v);
-        p.L[o] = kLn2 * (st.acc / st.l1 + (st.m2 - st.m1) + (lg2v - lg1));
+        if (p.nsplit > 1) {
+          // partial state of this key chunk, merged by streamkl_fwd_merge_kernel
+          const size_t rows = static_cast<size_t>(p.BH) * p.NQ;
+          float* dst = p.part + static_cast<size_t>(w.split) * 5 * rows + o;
+          dst[0 * rows] = st.m1;
+          dst[1 * rows] = st.m2;
+          dst[2 * rows] = st.l1;
+          dst[3 * rows] = st.l2;
+          dst[4 * rows] = st.acc;
+        } else if (nkt > 0) {
+          const float lg1 = lg2(st.l1), lg2v = lg2(st.l2);
+          p.LSE1[o] = kLn2 * (st.m1 + lg1);
+          p.LSE2[o] = kLn2 * (st.m2 + lg2v);
+          p.L[o] = kLn2 * (st.acc / st.l1 + (st.m2 - st.m1) + (lg2v - lg1));
+        }
       }
     }
   }
@@ -407,6 +431,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// Split-K merge (the page's Split-K variant, section 3): per row, combine the
+// partial states of the key chunks that overlap its visible keys,
+//   m = max_c m_c,  l = sum_c l_c 2^(m_c - m),  acc = sum_c acc_c 2^(m1_c - m1),
+// then finish as the unsplit kernel does.  acc_c holds sum p1 (y1 - y2) with p1
+// relative to m1_c, so it rescales with the teacher's factor.
+__global__ void streamkl_fwd_merge_kernel(const FwdMergeParams p) {
+  const long long rows = static_cast<long long>(p.BH) * p.NQ;
+  const int off = p.NK - p.NQ;
+  for (long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; r < rows;
+       r += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int i = static_cast<int>(r % p.NQ);
+    const int lim = p.causal ? min(p.NK, i + off + 1) : p.NK;
+    const int nc = min(p.nsplit, (lim + p.kt_chunk * BK - 1) / (p.kt_chunk * BK));
+    float m1 = -INFINITY, m2 = -INFINITY;
+    for (int c = 0; c < nc; ++c) {
+      m1 = fmaxf(m1, p.part[(static_cast<size_t>(c) * 5 + 0) * rows + r]);
+      m2 = fmaxf(m2, p.part[(static_cast<size_t>(c) * 5 + 1) * rows + r]);
+    }
+    float l1 = 0.f, l2 = 0.f, acc = 0.f;
+    for (int c = 0; c < nc; ++c) {
+      const float* q = p.part + static_cast<size_t>(c) * 5 * rows + r;
+      const float f1 = ex2(q[0] - m1), f2 = ex2(q[1 * rows] - m2);  // 0 for an empty chunk
+      l1 = fmaf(q[2 * rows], f1, l1);
+      l2 = fmaf(q[3 * rows], f2, l2);
+      acc = fmaf(q[4 * rows], f1, acc);
+    }
+    const float lg1 = lg2(l1), lg2v = lg2(l2);
+    p.LSE1[r] = kLn2 * (m1 + lg1);
+    p.LSE2[r] = kLn2 * (m2 + lg2v);
+    p.L[r] = kLn2 * (acc / l1 + (m2 - m1) + (lg2v - lg1));
   }
 }
 
@@ -428,6 +485,11 @@ size_t fwd_smem_bytes(int d1, int d2) {
   if (d1 == 64 && d2 == 128) return FwdLayout<64, 128>::alloc;
   if (d1 == 64 && d2 == 64) return FwdLayout<64, 64>::alloc;
   return 0;
+}
+
+cudaError_t launch_fwd_merge(const FwdMergeParams& p, int num_sms, cudaStream_t stream) {
+  streamkl_fwd_merge_kernel<<<num_sms * 4, 256, 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(const FwdParams& p, int d1, int d2, int grid, cudaStream_t stream) {

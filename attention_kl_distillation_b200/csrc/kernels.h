@@ -26,7 +26,22 @@ struct FwdParams {
   int* status;   // device status word
   unsigned long long wait_limit_ns;
   int withhold_keys;  // test hook: the producer issues no key tiles (waits then time out)
+  // Split-K: 0 = off.  Otherwise every unit covers key tiles [c*kt_chunk, (c+1)*kt_chunk)
+  // of split c < nsplit and writes its rows' partial states to `part`
+  // ([nsplit][5][BH*NQ]: m1, m2, l1, l2, acc in the base-2 domain) instead of L/LSE.
+  int kt_chunk, nsplit;
+  float* part;
 };
+
+struct FwdMergeParams {
+  const float* part;
+  float* L;
+  float* LSE1;
+  float* LSE2;
+  int BH, NQ, NK, causal, nsplit, kt_chunk;
+};
+
+cudaError_t launch_fwd_merge(const FwdMergeParams& p, int num_sms, cudaStream_t stream);
 
 // Dynamic shared memory the forward kernel needs for head dims (d1, d2).
 size_t fwd_smem_bytes(int d1, int d2);
@@ -103,9 +118,9 @@ cudaError_t launch_bwd_convert(const BwdConvertParams& p, int num_sms, cudaStrea
 
 __host__ __device__ inline int bwd_units(int BH, int NK) { return BH * ((NK + kBwdBK - 1) / kBwdBK); }
 
-// Work units of the forward: (bh, 256-row query block) pairs.
-__host__ __device__ inline int fwd_units(int BH, int NQ) {
-  return BH * ((NQ + kFwdBQ * kFwdTiles - 1) / (kFwdBQ * kFwdTiles));
+// Work units of the forward: (bh, 256-row query block) pairs, times the key splits.
+__host__ __device__ inline int fwd_units(int BH, int NQ, int nsplit = 1) {
+  return BH * ((NQ + kFwdBQ * kFwdTiles - 1) / (kFwdBQ * kFwdTiles)) * (nsplit > 1 ? nsplit : 1);
 }
 
 }  // namespace skl

@@ -274,46 +274,143 @@ streamkl_status streamkl_query_device_status(streamkl_stream_t stream) {
   return STREAMKL_EDEVICE;
 }
 
-streamkl_status streamkl_fwd(const streamkl_problem* prob, const void* Q1, const void* K1,
-                             const void* Q2, const void* K2, float* L, float* LSE1, float* LSE2,
-                             streamkl_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Validates forward arguments and fills the parameter block (maps, outputs,
+// scales, status word).  Split-K fields are left off.
+streamkl_status prepare_fwd(const streamkl_problem* prob, const void* Q1, const void* K1,
+                            const void* Q2, const void* K2, float* L, float* LSE1, float* LSE2,
+                            skl::FwdParams* p, DeviceInfo** devp) {
   streamkl_status st = check_problem(prob);
   if (st != STREAMKL_OK) return st;
   const void* ins[4] = {Q1, K1, Q2, K2};
-  for (const void* p : ins)
-    if (!p || !aligned16(p)) return STREAMKL_EINVAL;
+  for (const void* q : ins)
+    if (!q || !aligned16(q)) return STREAMKL_EINVAL;
   if (!L || !LSE1 || !LSE2) return STREAMKL_EINVAL;
   if ((reinterpret_cast<uintptr_t>(L) | reinterpret_cast<uintptr_t>(LSE1) |
        reinterpret_cast<uintptr_t>(LSE2)) & 3u)
     return STREAMKL_EINVAL;
-
   DeviceInfo* dev = nullptr;
   if ((st = current_device(&dev)) != STREAMKL_OK) return st;
-
   const int64_t BH = static_cast<int64_t>(prob->B) * prob->H;
+  if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, skl::kFwdBQ, &p->tmQ1)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kFwdBK, &p->tmK1)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, skl::kFwdBQ, &p->tmQ2)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(K2, BH, prob->NK, prob->d2, skl::kFwdBK, &p->tmK2)) != STREAMKL_OK) return st;
+  p->L = L;
+  p->LSE1 = LSE1;
+  p->LSE2 = LSE2;
+  p->BH = static_cast<int>(BH);
+  p->NQ = prob->NQ;
+  p->NK = prob->NK;
+  p->causal = prob->causal;
+  p->c1 = scale_or_default(prob->s1, prob->d1) * kLog2e;
+  p->c2 = scale_or_default(prob->s2, prob->d2) * kLog2e;
+  p->status = dev->status;
+  p->wait_limit_ns = wait_limit_ns();
+  p->withhold_keys = g_fault_mode.exchange(0) == 1 ? 1 : 0;
+  p->kt_chunk = 0;
+  p->nsplit = 1;
+  p->part = nullptr;
+  *devp = dev;
+  return STREAMKL_OK;
+}
+
+int fwd_key_tiles(const streamkl_problem& pr) { return (pr.NK + skl::kFwdBK - 1) / skl::kFwdBK; }
+
+// Key tiles per chunk and the effective chunk count for a requested split.
+void split_shape(const streamkl_problem& pr, int nsplit, int* kt_chunk, int* nsp) {
+  const int nkt = fwd_key_tiles(pr);
+  if (nsplit > nkt) nsplit = nkt;
+  if (nsplit < 1) nsplit = 1;
+  const int chunk = (nkt + nsplit - 1) / nsplit;
+  *kt_chunk = chunk;
+  *nsp = (nkt + chunk - 1) / chunk;
+}
+
+}  // namespace
+
+extern "C" {
+
+streamkl_status streamkl_fwd(const streamkl_problem* prob, const void* Q1, const void* K1,
+                             const void* Q2, const void* K2, float* L, float* LSE1, float* LSE2,
+                             streamkl_stream_t stream) {
   skl::FwdParams p;
-  if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, skl::kFwdBQ, &p.tmQ1)) != STREAMKL_OK) return st;
-  if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kFwdBK, &p.tmK1)) != STREAMKL_OK) return st;
-  if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, skl::kFwdBQ, &p.tmQ2)) != STREAMKL_OK) return st;
-  if ((st = tensor_map(K2, BH, prob->NK, prob->d2, skl::kFwdBK, &p.tmK2)) != STREAMKL_OK) return st;
-  p.L = L;
-  p.LSE1 = LSE1;
-  p.LSE2 = LSE2;
-  p.BH = static_cast<int>(BH);
-  p.NQ = prob->NQ;
-  p.NK = prob->NK;
-  p.causal = prob->causal;
-  p.c1 = scale_or_default(prob->s1, prob->d1) * kLog2e;
-  p.c2 = scale_or_default(prob->s2, prob->d2) * kLog2e;
-  p.status = dev->status;
-  p.wait_limit_ns = wait_limit_ns();
-  p.withhold_keys = g_fault_mode.exchange(0) == 1 ? 1 : 0;
+  DeviceInfo* dev = nullptr;
+  streamkl_status st = prepare_fwd(prob, Q1, K1, Q2, K2, L, LSE1, LSE2, &p, &dev);
+  if (st != STREAMKL_OK) return st;
   const int units = skl::fwd_units(p.BH, p.NQ);
   const int grid = units < dev->num_sms ? units : dev->num_sms;
   if (skl::launch_fwd(p, prob->d1, prob->d2, grid, reinterpret_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return STREAMKL_ECUDA;
   g_launches.fetch_add(1);
+  return STREAMKL_OK;
+}
+
+size_t streamkl_fwd_splitk_workspace_size(const streamkl_problem* prob, int nsplit) {
+  if (check_problem(prob) != STREAMKL_OK || nsplit < 1) return 0;
+  int chunk, nsp;
+  split_shape(*prob, nsplit, &chunk, &nsp);
+  const size_t rows = static_cast<size_t>(prob->B) * prob->H * static_cast<size_t>(prob->NQ);
+  return round256(static_cast<size_t>(nsp) * 5 * rows * sizeof(float));
+}
+
+int streamkl_fwd_splitk_suggest(const streamkl_problem* prob) {
+  if (check_problem(prob) != STREAMKL_OK) return 0;
+  DeviceInfo* dev = nullptr;
+  if (current_device(&dev) != STREAMKL_OK) return 0;
+  const int units = skl::fwd_units(prob->B * prob->H, prob->NQ);
+  const int want = 2 * dev->num_sms;
+  if (units >= dev->num_sms) return 1;
+  int n = (want + units - 1) / units;
+  const int nkt = fwd_key_tiles(*prob);
+  if (n > nkt) n = nkt;
+  return n < 1 ? 1 : n;
+}
+
+streamkl_status streamkl_fwd_splitk(const streamkl_problem* prob, const void* Q1, const void* K1,
+                                    const void* Q2, const void* K2, float* L, float* LSE1,
+                                    float* LSE2, int nsplit, void* workspace, size_t ws_bytes,
+                                    streamkl_stream_t stream) {
+  if (nsplit < 1) return STREAMKL_EINVAL;
+  const size_t need = streamkl_fwd_splitk_workspace_size(prob, nsplit);
+  if (need == 0) return check_problem(prob) != STREAMKL_OK ? check_problem(prob) : STREAMKL_EINVAL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need)
+    return STREAMKL_EINVAL;
+  skl::FwdParams p;
+  DeviceInfo* dev = nullptr;
+  streamkl_status st = prepare_fwd(prob, Q1, K1, Q2, K2, L, LSE1, LSE2, &p, &dev);
+  if (st != STREAMKL_OK) return st;
+  int chunk, nsp;
+  split_shape(*prob, nsplit, &chunk, &nsp);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (nsp > 1) {
+    p.kt_chunk = chunk;
+    p.nsplit = nsp;
+    p.part = static_cast<float*>(workspace);
+  }
+  const int units = skl::fwd_units(p.BH, p.NQ, p.nsplit);
+  const int grid = units < dev->num_sms ? units : dev->num_sms;
+  if (skl::launch_fwd(p, prob->d1, prob->d2, grid, s) != cudaSuccess) return STREAMKL_ECUDA;
+  g_launches.fetch_add(1);
+  if (nsp > 1) {
+    skl::FwdMergeParams mp;
+    mp.part = p.part;
+    mp.L = L;
+    mp.LSE1 = LSE1;
+    mp.LSE2 = LSE2;
+    mp.BH = p.BH;
+    mp.NQ = p.NQ;
+    mp.NK = p.NK;
+    mp.causal = p.causal;
+    mp.nsplit = nsp;
+    mp.kt_chunk = chunk;
+    if (skl::launch_fwd_merge(mp, dev->num_sms, s) != cudaSuccess) return STREAMKL_ECUDA;
+    g_launches.fetch_add(1);
+  }
   return STREAMKL_OK;
 }
 

@@ -79,6 +79,34 @@ streamkl_status streamkl_fwd(const streamkl_problem *prob, const void *Q1, const
                              streamkl_stream_t stream);
 
 /*
+ * Split-K forward (section 3, "Variante Split-K": for few query rows, e.g. a
+ * decode step with N_Q = 1, the keys are partitioned across thread blocks so
+ * that every SM has work).  Same results as streamkl_fwd within rounding.
+ * The keys of every 256-row query block are cut into `nsplit` chunks of equal
+ * length (in 64-key tiles); each chunk's blocks write partial row states
+ * (m1, m2, l1, l2, acc) to `workspace`, and a merge kernel combines them into
+ * L, LSE1, LSE2.  nsplit >= 1 (1 = no split); nsplit above the number of key
+ * tiles is clamped.  workspace: streamkl_fwd_splitk_workspace_size(prob,
+ * nsplit) bytes of device memory, 256-byte aligned, caller-owned; contents on
+ * entry do not matter.  Errors: as streamkl_fwd, plus EINVAL for nsplit < 1
+ * or a short/unaligned workspace.
+ */
+streamkl_status streamkl_fwd_splitk(const streamkl_problem *prob, const void *Q1, const void *K1,
+                                    const void *Q2, const void *K2, float *L, float *LSE1,
+                                    float *LSE2, int nsplit, void *workspace, size_t ws_bytes,
+                                    streamkl_stream_t stream);
+
+/* Workspace bytes for streamkl_fwd_splitk (0 on a bad problem or nsplit < 1). */
+size_t streamkl_fwd_splitk_workspace_size(const streamkl_problem *prob, int nsplit);
+
+/*
+ * A split count for the current device: enough key chunks that the forward's
+ * work units fill every SM about twice; 1 when the problem already does.
+ * 0 on a bad problem or if the device cannot be queried.
+ */
+int streamkl_fwd_splitk_suggest(const streamkl_problem *prob);
+
+/*
  * Workspace bytes that streamkl_bwd needs for this problem: an fp32 dQ
  * accumulator [B][H][NQ][d1+d2] (section 2, "Fusione del Kernel": dQ is
  * accumulated with atomics across key tiles) plus padding.  0 on a bad

@@ -123,3 +123,17 @@ def test_bwd_algorithm_selection():
         assert B.bwd_algorithm_for(4, 32, 65536, 65536, 128, 128, True) == "split"
     finally:
         B.set_bwd_algorithm("auto")
+
+
+def test_splitk_workspace_and_validation():
+    assert B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 3) >= 3 * 5 * 2 * 10 * 4
+    assert B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 0) == 0
+    # nsplit beyond the 10 key tiles is clamped
+    assert B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 50) == B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 10)
+    lib = B.lib()
+    prob = B.problem(1, 2, 10, 640, 64, 64)
+    v = ctypes.c_void_p
+    args = [v(16 * (k + 1)) for k in range(7)]
+    assert lib.streamkl_fwd_splitk(ctypes.byref(prob), *args, 0, v(1 << 20), 1 << 30, v(0)) == B.EINVAL
+    assert lib.streamkl_fwd_splitk(ctypes.byref(prob), *args, 2, v(0), 1 << 30, v(0)) == B.EINVAL
+    assert lib.streamkl_fwd_splitk(ctypes.byref(prob), *args, 2, v(1 << 20), 8, v(0)) == B.EINVAL
