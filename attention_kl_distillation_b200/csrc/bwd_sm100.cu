@@ -359,6 +359,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       constexpr uint32_t idQ1 = idesc_bf16(D1, BQ, 1, 1);         // dQ1^T: A = K1 MN-major
       constexpr uint32_t idQ2 = idesc_bf16(D2, BQ, 1, 1);
       const uint32_t k1a = smem_u32(k1_s), k2a = smem_u32(k2_s);
+      const uint64_t k1d = sdesc_sw128(k1a, 16, 1024), k2d = sdesc_sw128(k2a, 16, 1024);
+      // K tiles read MN-major for dQ^T: 64-feature chunks 16 KB apart
+      const uint64_t k1m = sdesc_sw128(k1a, BK * 128, 1024), k2m = sdesc_sw128(k2a, BK * 128, 1024);
       int us = 0, qs_s = 0, qs_r = 0, db = 0;
       uint32_t uph = 0, kph = 0, qph_s = 0, sph = 0, dkph = 0;
       uint32_t dqph[2] = {0, 0};
@@ -380,20 +383,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           if (!mbar_wait(&qfull[qs_s], qph_s, ctl)) return false;
           if (!mbar_wait(sempty, sph ^ 1, ctl)) return false;
           tc_fence_after();
-          const uint32_t qa1 = smem_u32(q1_s(qs_s)), qa2 = smem_u32(q2_s(qs_s));
+          const uint64_t q1d = sdesc_sw128(smem_u32(q1_s(qs_s)), 16, 1024);
+          const uint64_t q2d = sdesc_sw128(smem_u32(q2_s(qs_s)), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D1 / 16; ++kk) {
             const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(tmem_base + kColS1,
-                         sdesc_sw128(k1a + (kk >> 2) * (BK * 128) + o, 16, 1024),
-                         sdesc_sw128(qa1 + (kk >> 2) * (BQ * 128) + o, 16, 1024), idS, kk > 0);
+            umma_bf16_ss(tmem_base + kColS1, sdesc_advance(k1d, (kk >> 2) * (BK * 128) + o),
+                         sdesc_advance(q1d, (kk >> 2) * (BQ * 128) + o), idS, kk > 0);
           }
 #pragma unroll
           for (int kk = 0; kk < D2 / 16; ++kk) {
             const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(tmem_base + kColS2,
-                         sdesc_sw128(k2a + (kk >> 2) * (BK * 128) + o, 16, 1024),
-                         sdesc_sw128(qa2 + (kk >> 2) * (BQ * 128) + o, 16, 1024), idS, kk > 0);
+            umma_bf16_ss(tmem_base + kColS2, sdesc_advance(k2d, (kk >> 2) * (BK * 128) + o),
+                         sdesc_advance(q2d, (kk >> 2) * (BQ * 128) + o), idS, kk > 0);
           }
           umma_commit(sfull);
           sph ^= 1;
@@ -413,18 +415,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
             dkph ^= 1;
           }
           tc_fence_after();
-          const uint32_t qa1 = smem_u32(q1_s(qs_r)), qa2 = smem_u32(q2_s(qs_r));
-          const uint32_t d1a = smem_u32(ds1_s(db)), d2a = smem_u32(ds2_s(db));
+          // dS^T tiles read K-major for dK and MN-major for dQ^T; Q tiles MN-major for dK
+          const uint64_t q1m = sdesc_sw128(smem_u32(q1_s(qs_r)), BQ * 128, 1024);
+          const uint64_t q2m = sdesc_sw128(smem_u32(q2_s(qs_r)), BQ * 128, 1024);
+          const uint64_t d1k = sdesc_sw128(smem_u32(ds1_s(db)), 16, 1024);
+          const uint64_t d2k = sdesc_sw128(smem_u32(ds2_s(db)), 16, 1024);
+          const uint64_t d1m = sdesc_sw128(smem_u32(ds1_s(db)), BQ * 128, 1024);
+          const uint64_t d2m = sdesc_sw128(smem_u32(ds2_s(db)), BQ * 128, 1024);
           // dK_t += (s_t dS_t)^T Q_t : A = dS^T (K-major, 128B rows of 64 queries),
           // B = Q_t read MN-major (features contiguous; 64-feature chunks 8 KB apart).
 #pragma unroll
           for (int kk = 0; kk < BQ / 16; ++kk) {
             if (p.want_dk1)
-              umma_bf16_ss(tmem_base + kColDK1, sdesc_sw128(d1a + kk * 32, 16, 1024),
-                           sdesc_sw128(qa1 + kk * 2048, BQ * 128, 1024), idK1, (t > 0 || kk > 0));
+              umma_bf16_ss(tmem_base + kColDK1, sdesc_sw128(smem_u32(ds1_s(db)) + kk * 32, 16, 1024),
+                           sdesc_sw128(smem_u32(q1_s(qs_r)) + kk * 2048, BQ * 128, 1024), idK1, (t > 0 || kk > 0));
             if (p.want_dk2)
-              umma_bf16_ss(tmem_base + kColDK1 + D1, sdesc_sw128(d2a + kk * 32, 16, 1024),
-                           sdesc_sw128(qa2 + kk * 2048, BQ * 128, 1024), idK2, (t > 0 || kk > 0));
+              umma_bf16_ss(tmem_base + kColDK1 + D1, sdesc_sw128(smem_u32(ds2_s(db)) + kk * 32, 16, 1024),
+                           sdesc_sw128(smem_u32(q2_s(qs_r)) + kk * 2048, BQ * 128, 1024), idK2, (t > 0 || kk > 0));
           }
           // dQ_t^T = K_t^T (s_t dS_t)^T : A = K tile read MN-major (64-feature chunks
           // 16 KB apart), B = dS^T read MN-major (64 queries contiguous per key).
@@ -434,8 +441,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           if (p.want_dq1) {
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              umma_bf16_ss(tmem_base + kColDQ1, sdesc_sw128(k1a + kk * 2048, BK * 128, 1024),
-                           sdesc_sw128(d1a + kk * 2048, BQ * 128, 1024), idQ1, kk > 0);
+              umma_bf16_ss(tmem_base + kColDQ1, sdesc_advance(k1m, kk * 2048),
+                           sdesc_advance(d1m, kk * 2048), idQ1, kk > 0);
           }
           if (!(ok = mbar_wait(&dqempty[1], dqph[1] ^ 1, ctl))) break;
           dqph[1] ^= 1;
@@ -443,8 +450,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           if (p.want_dq2) {
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              umma_bf16_ss(tmem_base + kColDQ2, sdesc_sw128(k2a + kk * 2048, BK * 128, 1024),
-                           sdesc_sw128(d2a + kk * 2048, BQ * 128, 1024), idQ2, kk > 0);
+              umma_bf16_ss(tmem_base + kColDQ2, sdesc_advance(k2m, kk * 2048),
+                           sdesc_advance(d2m, kk * 2048), idQ2, kk > 0);
           }
           umma_commit(dqfull);
           umma_commit(&dsempty[db]);

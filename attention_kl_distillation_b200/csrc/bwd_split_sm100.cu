@@ -320,7 +320,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr uint32_t idS = idesc_bf16(RB, CB);         // S: M=128 resident, N=64 streamed
       constexpr uint32_t idO1 = idesc_bf16(RB, D1, 0, 1);  // OUT1: A = dS (TMEM), B = C1 MN-major
       constexpr uint32_t idO2 = idesc_bf16(RB, D2, 0, 1);
-      const uint32_t r1a = smem_u32(r1_s), r2a = smem_u32(r2_s);
+      const uint64_t r1d = sdesc_sw128(smem_u32(r1_s), 16, 1024);
+      const uint64_t r2d = sdesc_sw128(smem_u32(r2_s), 16, 1024);
       int us = 0, cs_s = 0, cs_r = 0, db = 0;
       uint32_t uph = 0, rph = 0, cph_s = 0, sph = 0, oph = 0;
       uint32_t dsph[2] = {0, 0};
@@ -341,20 +342,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!mbar_wait(&cfull[cs_s], cph_s, ctl)) return false;
           if (!mbar_wait(sempty, sph ^ 1, ctl)) return false;
           tc_fence_after();
-          const uint32_t ca1 = smem_u32(c1_s(cs_s)), ca2 = smem_u32(c2_s(cs_s));
+          const uint64_t c1d = sdesc_sw128(smem_u32(c1_s(cs_s)), 16, 1024);
+          const uint64_t c2d = sdesc_sw128(smem_u32(c2_s(cs_s)), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D1 / 16; ++kk) {
             const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(tmem_base + kColS1,
-                         sdesc_sw128(r1a + (kk >> 2) * (RB * 128) + o, 16, 1024),
-                         sdesc_sw128(ca1 + (kk >> 2) * (CB * 128) + o, 16, 1024), idS, kk > 0);
+            umma_bf16_ss(tmem_base + kColS1, sdesc_advance(r1d, (kk >> 2) * (RB * 128) + o),
+                         sdesc_advance(c1d, (kk >> 2) * (CB * 128) + o), idS, kk > 0);
           }
 #pragma unroll
           for (int kk = 0; kk < D2 / 16; ++kk) {
             const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(tmem_base + kColS2,
-                         sdesc_sw128(r2a + (kk >> 2) * (RB * 128) + o, 16, 1024),
-                         sdesc_sw128(ca2 + (kk >> 2) * (CB * 128) + o, 16, 1024), idS, kk > 0);
+            umma_bf16_ss(tmem_base + kColS2, sdesc_advance(r2d, (kk >> 2) * (RB * 128) + o),
+                         sdesc_advance(c2d, (kk >> 2) * (CB * 128) + o), idS, kk > 0);
           }
           umma_commit(sfull);
           sph ^= 1;
@@ -374,18 +374,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             oph ^= 1;
           }
           tc_fence_after();
-          const uint32_t ca1 = smem_u32(c1_s(cs_r)), ca2 = smem_u32(c2_s(cs_r));
+          // C tiles read MN-major: features contiguous, 64-feature chunks 8 KB apart
+          const uint64_t c1m = sdesc_sw128(smem_u32(c1_s(cs_r)), CB * 128, 1024);
+          const uint64_t c2m = sdesc_sw128(smem_u32(c2_s(cs_r)), CB * 128, 1024);
           const uint32_t dsa = tmem_base + kColDS + db * 64;
           // OUT_t += dS_t (TMEM, 64 streamed rows along K, 8 columns per 16) . C_t
           // (read MN-major: features contiguous, 64-feature chunks 8 KB apart).
 #pragma unroll
           for (int kk = 0; kk < CB / 16; ++kk) {
             if (p.out1)
-              umma_bf16_ts(tmem_base + kColOut, dsa + kk * 8,
-                           sdesc_sw128(ca1 + kk * 2048, CB * 128, 1024), idO1, (t > 0 || kk > 0));
+              umma_bf16_ts(tmem_base + kColOut, dsa + kk * 8, sdesc_advance(c1m, kk * 2048), idO1,
+                           (t > 0 || kk > 0));
             if (p.out2)
-              umma_bf16_ts(tmem_base + kColOut + D1, dsa + 32 + kk * 8,
-                           sdesc_sw128(ca2 + kk * 2048, CB * 128, 1024), idO2, (t > 0 || kk > 0));
+              umma_bf16_ts(tmem_base + kColOut + D1, dsa + 32 + kk * 8, sdesc_advance(c2m, kk * 2048),
+                           idO2, (t > 0 || kk > 0));
           }
           umma_commit(&dsempty[db]);
           umma_commit(&cempty[cs_r]);

@@ -8,21 +8,27 @@
 // B200 mapping (one CTA per SM, persistent):
 //   work unit   (bh, 256-row query block) = two 128-row tiles A and B that
 //               share every key tile, so each K tile is read once per 256 rows
-//   warp 0      TMA producer: Q1/Q2 for both tiles once per unit, K1/K2 tiles
-//               into a shared-memory ring (128-byte swizzle, no multicast)
+//   warp 0      TMA producer: K1/K2 tiles into a ring of up to six stages
+//               (128-byte swizzle, no multicast)
 //   warp 1      TMEM owner and UMMA issuer: per key tile and query tile,
 //               S1 = Q1 K1^T and S2 = Q2 K2^T (tcgen05.mma kind::f16, fp32
-//               accumulators) into that tile's double-buffered TMEM slot
-//   warps 2..5  reduction warpgroup of tile A, warps 6..9 of tile B: thread r
-//               owns query row r (TMEM lane r), loads its 64 + 64 logits with
-//               tcgen05.ld, frees the slot and applies the online update in
-//               registers: exp2 on the MUFU pipe, the softmax scale folded into
-//               the exponent argument, packed f32x2 arithmetic elsewhere.
-//               Two warpgroups put two reduction warps on every SM sub-partition
-//               so that one hides the other's latencies.
+//               accumulators).  Q lives in TMEM as the A operand, K in shared
+//               memory as B; keeping Q out of shared memory is what leaves room
+//               for a ring deep enough to cover the TMA latency.
+//   warps 2..17 four reduction warpgroups, two per query tile, each owning 32
+//               of the 64 keys of every key tile: thread r owns query row r
+//               (TMEM lane r).  At the start of a unit it copies its row of Q1
+//               (first warpgroup) or Q2 (second) from global memory into TMEM;
+//               per key tile it loads its 32 + 32 logits with tcgen05.ld, frees
+//               the slot and applies the online update in registers (exp2 on
+//               the MUFU pipe, the softmax scale folded into the exponent
+//               argument, packed f32x2 arithmetic elsewhere).  The two key halves
+//               of a row keep separate running states and merge at the end of the
+//               unit.  Four reduction warps per SM sub-partition hide each
+//               other's latencies.
 // The accumulator acc is one fp32 per row: there is no PV product and no
-// output tile, which is what lets both S tiles of both query tiles live in
-// TMEM (4 x 128 of the 512 columns) at once.
+// output tile.  TMEM: S1/S2 of tile A [0,128), of tile B [128,256); Q1/Q2 of
+// tile A and tile B as bf16 A operands [256, 256 + d1 + d2).
 //
 // Units are visited longest first (the last query blocks of a causal problem
 // see the most keys) and dealt to CTAs in a snake order, an approximation of
@@ -39,32 +45,35 @@ namespace {
 constexpr int BQ = kFwdBQ;
 constexpr int NT = kFwdTiles;
 constexpr int BK = kFwdBK;
-constexpr int SBUF = 2;  // TMEM S1/S2 slots per query tile
-constexpr int NTHREADS = 64 + NT * 128;
+constexpr int NH = 2;    // reduction warpgroups per query tile, each owning BK/NH keys of a tile
+constexpr int KH = BK / NH;
+constexpr int NTHREADS = 64 + NT * NH * 128;
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D1, int D2>
 struct FwdLayout {
-  static constexpr int q1_tile = BQ * D1 * 2;
-  static constexpr int q2_tile = BQ * D2 * 2;
   static constexpr int k1_bytes = BK * D1 * 2;
   static constexpr int k2_bytes = BK * D2 * 2;
   static constexpr int stage_bytes = k1_bytes + k2_bytes;
-  static constexpr int q_bytes = NT * (q1_tile + q2_tile);
-  static constexpr int KSTAGES = (q_bytes + 4 * stage_bytes + 2048 <= 232448) ? 4 : 3;
-  static constexpr int q1_off = 0;
-  static constexpr int q2_off = q1_off + NT * q1_tile;
-  static constexpr int k_off = q2_off + NT * q2_tile;
+  static constexpr int handover_bytes = NT * 5 * BQ * 4;
+  static constexpr int ks_fit = (232448 - 1024 - 512 - handover_bytes) / stage_bytes;
+  static constexpr int KSTAGES = ks_fit > 6 ? 6 : ks_fit;
+  static constexpr int k_off = 0;
   static constexpr int bar_off = k_off + KSTAGES * stage_bytes;
-  // barriers: qfull, qempty, kfull[KS], kempty[KS], sfull[NT][SBUF], sempty[NT][SBUF], drain
-  static constexpr int nbar = 3 + 2 * KSTAGES + 2 * NT * SBUF;
+  // barriers: qready[NT], qfree[NT], kfull[KS], kempty[KS], sfull[NT], sempty[NT], drain
+  static constexpr int nbar = 1 + 2 * KSTAGES + 4 * NT;
   static constexpr int misc_off = bar_off + nbar * 8;
-  static constexpr int total = misc_off + 16;
+  static constexpr int part_off = misc_off + 16;  // key-half partial states [NT][5][BQ] fp32
+  static constexpr int total = part_off + handover_bytes;
   static constexpr int alloc = total + 1024;  // slack to align the base to 1024 B
+  static_assert(KSTAGES >= 3, "key ring too shallow");
   static_assert(alloc <= 232448, "shared memory budget exceeded");
-  static_assert(q1_tile % 1024 == 0 && q2_tile % 1024 == 0 && k1_bytes % 1024 == 0 &&
-                    k2_bytes % 1024 == 0,
+  static_assert(k1_bytes % 1024 == 0 && k2_bytes % 1024 == 0,
                 "tiles must keep 1024-byte alignment for the 128B swizzle atoms");
+  // TMEM columns
+  __host__ __device__ static constexpr uint32_t s_col(int t) { return t * 2 * BK; }          // S1; S2 at +BK
+  __host__ __device__ static constexpr uint32_t q_col(int t) { return NT * 2 * BK + t * (D1 + D2) / 2; }  // Q1; Q2 at +D1/2
+  static_assert(NT * 2 * BK + NT * (D1 + D2) / 2 <= 512, "TMEM budget exceeded");
 };
 
 struct Sched {
@@ -130,17 +139,18 @@ struct RowState {
   float m1, m2, l1, l2, acc;
 };
 
-// One key tile of the online update for one row.  a/b hold the raw fp32
-// products <Q1_i, K1_j> and <Q2_i, K2_j>; c1/c2 fold the softmax scale and
-// log2(e).  With MASK, only the first nv keys of the tile are visible.
+// One key tile (this warpgroup's KH keys of it) of the online update for one
+// row.  a/b hold the raw fp32 products <Q1_i, K1_j> and <Q2_i, K2_j>; c1/c2
+// fold the softmax scale and log2(e).  With MASK, only the first nv keys are
+// visible.
 template <bool MASK>
-__device__ __forceinline__ void tile_update(const uint32_t (&a)[BK], const uint32_t (&b)[BK],
+__device__ __forceinline__ void tile_update(const uint32_t (&a)[KH], const uint32_t (&b)[KH],
                                             float c1, float c2, int nv, RowState& st) {
   float mx1[4], mx2[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) mx1[k] = mx2[k] = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < BK; j += 2) {
+  for (int j = 0; j < KH; j += 2) {
     float v1a = __uint_as_float(a[j]), v1b = __uint_as_float(a[j + 1]);
     float v2a = __uint_as_float(b[j]), v2b = __uint_as_float(b[j + 1]);
     if (MASK) {
@@ -166,7 +176,7 @@ __device__ __forceinline__ void tile_update(const uint32_t (&a)[BK], const uint3
 #pragma unroll
   for (int k = 0; k < 2; ++k) sp1[k] = sp2[k] = sd[k] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int j = 0; j < BK; j += 2) {
+  for (int j = 0; j < KH; j += 2) {
     const float2 v1 = make_float2(__uint_as_float(a[j]), __uint_as_float(a[j + 1]));
     const float2 v2 = make_float2(__uint_as_float(b[j]), __uint_as_float(b[j + 1]));
     float2 t1 = __ffma2_rn(v1, C1, M1);  // log2 of the unnormalised teacher weight
@@ -195,6 +205,30 @@ __device__ __forceinline__ void tile_update(const uint32_t (&a)[BK], const uint3
   st.m2 = m2n;
 }
 
+// Copies query row `row` of Q ([BH][NQ][D] bf16) into TMEM columns [col,
+// col + D/2) of this thread's lane as the A operand of the S products (two
+// features per 32-bit column, the lower feature in the low half); rows past
+// NQ are zero.
+template <int D>
+__device__ __forceinline__ void stage_q_row(const __nv_bfloat16* Q, int bh, int NQ, int row,
+                                            uint32_t taddr) {
+  const bool ok = row < NQ;
+  const uint4* src = reinterpret_cast<const uint4*>(Q + (static_cast<size_t>(bh) * NQ + (ok ? row : 0)) * D);
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {  // 32 features = 16 columns per chunk
+    uint32_t v[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint4 x = ok ? __ldg(src + c * 4 + k) : make_uint4(0u, 0u, 0u, 0u);
+      v[4 * k + 0] = x.x;
+      v[4 * k + 1] = x.y;
+      v[4 * k + 2] = x.z;
+      v[4 * k + 3] = x.w;
+    }
+    tmem_st_32x32b_x16(taddr + c * 16, v);
+  }
+}
+
 template <int D1, int D2>
 __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_constant__ FwdParams p) {
   using Lay = FwdLayout<D1, D2>;
@@ -203,13 +237,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off);
-  uint64_t* qfull = bars + 0;
-  uint64_t* qempty = bars + 1;
-  uint64_t* kfull = bars + 2;
+  uint64_t* qready = bars + 0;    // [NT]: the tile's Q rows of this unit are in TMEM
+  uint64_t* qfree = qready + NT;  // [NT]: the UMMAs of the previous unit have read them
+  uint64_t* kfull = qfree + NT;
   uint64_t* kempty = kfull + KS;
-  uint64_t* sfull = kempty + KS;      // [NT][SBUF]
-  uint64_t* sempty = sfull + NT * SBUF;
-  uint64_t* drain = sempty + NT * SBUF;
+  uint64_t* sfull = kempty + KS;  // [NT]
+  uint64_t* sempty = sfull + NT;  // [NT]
+  uint64_t* drain = sempty + NT;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::misc_off + 4);
 
@@ -219,21 +253,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(qfull, 1);
-    mbar_init(qempty, 1);
+    for (int t = 0; t < NT; ++t) {
+      mbar_init(&qready[t], 4 * NH);  // every reduction warp of the tile wrote its Q rows
+      mbar_init(&qfree[t], 1);
+    }
     for (int s = 0; s < KS; ++s) {
       mbar_init(&kfull[s], 1);
       mbar_init(&kempty[s], 1);
     }
-    for (int s = 0; s < NT * SBUF; ++s) {
-      mbar_init(&sfull[s], 1);
-      mbar_init(&sempty[s], 4);  // one arrival per reduction warp of that tile
+    for (int t = 0; t < NT; ++t) {
+      mbar_init(&sfull[t], 1);
+      mbar_init(&sempty[t], 4 * NH);  // one arrival per reduction warp of that tile
     }
     mbar_init(drain, 1);
     fence_mbar_init();
-    tma_prefetch_desc(&p.tmQ1);
     tma_prefetch_desc(&p.tmK1);
-    tma_prefetch_desc(&p.tmQ2);
     tma_prefetch_desc(&p.tmK2);
   }
   if (warp == 1) {
@@ -247,8 +281,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
 
   Sched sched{fwd_units(p.BH, p.NQ, p.nsplit), static_cast<int>(gridDim.x),
               static_cast<int>(blockIdx.x), 0};
-  auto q1_s = [&](int t) { return smem + Lay::q1_off + t * Lay::q1_tile; };
-  auto q2_s = [&](int t) { return smem + Lay::q2_off + t * Lay::q2_tile; };
   auto k1_s = [&](int s) { return smem + Lay::k_off + s * Lay::stage_bytes; };
   auto k2_s = [&](int s) { return smem + Lay::k_off + s * Lay::stage_bytes + Lay::k1_bytes; };
 
@@ -256,26 +288,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int ks = 0;
-      uint32_t kph = 0, qph = 0;
-      uint32_t armed_q = 0, armed_k[KS] = {};  // last armed phase + 1 (0 = never)
+      uint32_t kph = 0;
+      uint32_t armed_k[KS] = {};  // last armed phase + 1 (0 = never)
       int u;
       bool ok = true;
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
         if (w.nkt_max <= w.kt_lo) continue;  // split chunk past every row's frontier
-        if (!(ok = mbar_wait(qempty, qph ^ 1, ctl))) break;
-        mbar_arrive_expect_tx(qfull, Lay::q_bytes);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-#pragma unroll
-          for (int b = 0; b < D1 / 64; ++b)
-            tma_load_3d(q1_s(t) + b * (BQ * 128), &p.tmQ1, qfull, b * 64, w.q0 + t * BQ, w.bh);
-#pragma unroll
-          for (int b = 0; b < D2 / 64; ++b)
-            tma_load_3d(q2_s(t) + b * (BQ * 128), &p.tmQ2, qfull, b * 64, w.q0 + t * BQ, w.bh);
-        }
-        armed_q = qph + 1;
-        qph ^= 1;
         for (int kt = w.kt_lo; kt < (p.withhold_keys ? w.kt_lo : w.nkt_max); ++kt) {
           if (!(ok = mbar_wait(&kempty[ks], kph ^ 1, ctl))) break;
           mbar_arrive_expect_tx(&kfull[ks], Lay::stage_bytes);
@@ -296,7 +315,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
         // Aborting: let the copies already in flight land before the CTA exits.
         volatile int zero = 0;
         WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
-        if (armed_q) mbar_wait(qfull, armed_q - 1, dctl);
         for (int s = 0; s < KS; ++s)
           if (armed_k[s]) mbar_wait(&kfull[s], armed_k[s] - 1, dctl);
       }
@@ -306,7 +324,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(BQ, BK);
       int ks = 0;
-      int sb[NT] = {};
       uint32_t kph = 0, qph = 0;
       uint32_t sph[NT] = {};
       int u;
@@ -314,37 +331,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
         if (w.nkt_max <= w.kt_lo) continue;
-        if (!(ok = mbar_wait(qfull, qph, ctl))) break;
+#pragma unroll
+        for (int t = 0; t < NT; ++t)  // Q of this unit is in TMEM
+          if (ok) ok = mbar_wait(&qready[t], qph, ctl);
+        if (!ok) break;
         qph ^= 1;
         tc_fence_after();
         for (int kt = w.kt_lo; kt < w.nkt_max && ok; ++kt) {
           if (!(ok = mbar_wait(&kfull[ks], kph, ctl))) break;
-          const uint32_t k1a = smem_u32(k1_s(ks)), k2a = smem_u32(k2_s(ks));
+          // Descriptors built once per stage; each UMMA below costs an add and the
+          // MMA itself, so this thread keeps up although it shares its SM
+          // sub-partition with four busy reduction warps.
+          const uint64_t b1 = sdesc_sw128(smem_u32(k1_s(ks)), 16, 1024);
+          const uint64_t b2 = sdesc_sw128(smem_u32(k2_s(ks)), 16, 1024);
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
             if (kt >= w.nkt[t]) continue;
-            if (!(ok = mbar_wait(&sempty[t * SBUF + sb[t]], sph[t] ^ 1, ctl))) break;
+            if (!(ok = mbar_wait(&sempty[t], sph[t] ^ 1, ctl))) break;
+            sph[t] ^= 1;
             tc_fence_after();
-            const uint32_t q1a = smem_u32(q1_s(t)), q2a = smem_u32(q2_s(t));
-            const uint32_t t1 = tmem_base + (t * SBUF + sb[t]) * (2 * BK);
-            const uint32_t t2 = t1 + BK;
+            const uint32_t d1 = tmem_base + Lay::s_col(t), d2 = d1 + BK;
+            const uint32_t a1 = tmem_base + Lay::q_col(t), a2 = a1 + D1 / 2;
 #pragma unroll
-            for (int kk = 0; kk < D1 / 16; ++kk) {
-              const uint32_t o = (kk & 3) * 32;
-              umma_bf16_ss(t1, sdesc_sw128(q1a + (kk >> 2) * (BQ * 128) + o, 16, 1024),
-                           sdesc_sw128(k1a + (kk >> 2) * (BK * 128) + o, 16, 1024), idesc, kk > 0);
-            }
+            for (int kk = 0; kk < D1 / 16; ++kk)
+              umma_bf16_ts(d1, a1 + kk * 8,
+                           sdesc_advance(b1, (kk >> 2) * (BK * 128) + (kk & 3) * 32), idesc, kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < D2 / 16; ++kk) {
-              const uint32_t o = (kk & 3) * 32;
-              umma_bf16_ss(t2, sdesc_sw128(q2a + (kk >> 2) * (BQ * 128) + o, 16, 1024),
-                           sdesc_sw128(k2a + (kk >> 2) * (BK * 128) + o, 16, 1024), idesc, kk > 0);
-            }
-            umma_commit(&sfull[t * SBUF + sb[t]]);
-            if (++sb[t] == SBUF) {
-              sb[t] = 0;
-              sph[t] ^= 1;
-            }
+            for (int kk = 0; kk < D2 / 16; ++kk)
+              umma_bf16_ts(d2, a2 + kk * 8,
+                           sdesc_advance(b2, (kk >> 2) * (BK * 128) + (kk & 3) * 32), idesc, kk > 0);
+            umma_commit(&sfull[t]);
           }
           if (!ok) break;
           umma_commit(&kempty[ks]);
@@ -353,7 +369,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
             kph ^= 1;
           }
         }
-        if (ok) umma_commit(qempty);
+        if (!ok) break;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) umma_commit(&qfree[t]);  // once this unit's UMMAs are done
       }
       // Every UMMA issued by this thread completes before TMEM is released.
       umma_commit(drain);
@@ -363,48 +381,79 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     }
   } else {
     // ------------------------------------------------------------ reduction
-    const int t = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int rw = (warp - 2) >> 2;
+    const int t = rw / NH;   // query tile of this warpgroup
+    const int hf = rw % NH;  // which KH keys of every key tile it owns
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t tlane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    float* part = reinterpret_cast<float*>(smem + Lay::part_off) + t * 5 * BQ;
     const int off = p.NK - p.NQ;
-    int sb = 0;
-    uint32_t sph = 0;
+    uint32_t sph = 0, qfph = 0;
     int u;
     bool ok = true;
     while (ok && sched.next(u)) {
       const Unit w = decode_unit(p, u);
       if (w.nkt_max <= w.kt_lo) continue;
       const int i_abs = w.q0 + t * BQ + row;
+      // This unit's Q rows into TMEM, once the previous unit's UMMAs have read them.
+      if (!(ok = mbar_wait(&qfree[t], qfph ^ 1, ctl))) break;
+      qfph ^= 1;
+      tc_fence_after();
+      if (hf == 0)
+        stage_q_row<D1>(p.Q1, w.bh, p.NQ, i_abs, tlane + Lay::q_col(t));
+      else
+        stage_q_row<D2>(p.Q2, w.bh, p.NQ, i_abs, tlane + Lay::q_col(t) + D1 / 2);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qready[t]);
       const int lim = p.causal ? min(p.NK, i_abs + off + 1) : p.NK;  // visible keys [0, lim)
       RowState st{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
       const int nkt = w.nkt[t];
       for (int kt = w.kt_lo; kt < nkt; ++kt) {
-        if (!(ok = mbar_wait(&sfull[t * SBUF + sb], sph, ctl))) break;
+        if (!(ok = mbar_wait(&sfull[t], sph, ctl))) break;
+        sph ^= 1;
         tc_fence_after();
-        uint32_t a[BK], b[BK];
-        const uint32_t tcol = tlane + (t * SBUF + sb) * (2 * BK);
-        tmem_ld_32x32b_x32(tcol + 0, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-        tmem_ld_32x32b_x32(tcol + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-        tmem_ld_32x32b_x32(tcol + BK, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
-        tmem_ld_32x32b_x32(tcol + BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
+        uint32_t a[KH], b[KH];
+        const uint32_t tcol = tlane + Lay::s_col(t) + hf * KH;
+        tmem_ld_32x32b<KH>(tcol, a);
+        tmem_ld_32x32b<KH>(tcol + BK, b);
         tmem_ld_wait();
         reg_fence(a);
         reg_fence(b);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sempty[t * SBUF + sb]);
-        if (++sb == SBUF) {
-          sb = 0;
-          sph ^= 1;
-        }
+        if (lane == 0) mbar_arrive(&sempty[t]);
         if (kt >= w.kt_mask[t])
-          tile_update<true>(a, b, p.c1, p.c2, lim - kt * BK, st);
+          tile_update<true>(a, b, p.c1, p.c2, lim - kt * BK - hf * KH, st);
         else
-          tile_update<false>(a, b, p.c1, p.c2, BK, st);
+          tile_update<false>(a, b, p.c1, p.c2, KH, st);
       }
       if (!ok) break;
-      if (i_abs < p.NQ && w.q0 + t * BQ < p.NQ) {
+      // Merge the key halves of every row (same rescaling as the split-K merge):
+      // the second warpgroup hands its state over through shared memory.
+      if (hf == 1) {
+        part[0 * BQ + row] = st.m1;
+        part[1 * BQ + row] = st.m2;
+        part[2 * BQ + row] = st.l1;
+        part[3 * BQ + row] = st.l2;
+        part[4 * BQ + row] = st.acc;
+      }
+      named_bar_sync(1 + t, NH * 128);
+      if (hf == 0) {
+        const float om1 = part[0 * BQ + row], om2 = part[1 * BQ + row];
+        const float m1 = fmaxf(st.m1, om1), m2 = fmaxf(st.m2, om2);
+        const float fa1 = ex2(st.m1 - m1), fb1 = ex2(om1 - m1);  // 0 for a half with no key
+        const float fa2 = ex2(st.m2 - m2), fb2 = ex2(om2 - m2);
+        st.l1 = fmaf(st.l1, fa1, part[2 * BQ + row] * fb1);
+        st.l2 = fmaf(st.l2, fa2, part[3 * BQ + row] * fb2);
+        st.acc = fmaf(st.acc, fa1, part[4 * BQ + row] * fb1);
+        st.m1 = m1;
+        st.m2 = m2;
+      }
+      named_bar_sync(1 + t, NH * 128);  // the handover slot may be reused
+      if (hf == 0 && i_abs < p.NQ && w.q0 + t * BQ < p.NQ) {
         const size_t o = static_cast<size_t>(w.bh) * p.NQ + i_abs;
         if (p.nsplit > 1) {
           // partial state of this key chunk, merged by streamkl_fwd_merge_kernel

@@ -17,7 +17,9 @@ constexpr int kFwdTiles = 2;
 constexpr int kFwdBK = 64;
 
 struct FwdParams {
-  CUtensorMap tmQ1, tmK1, tmQ2, tmK2;  // 3-D maps over [BH][N][d], 128B swizzle
+  CUtensorMap tmK1, tmK2;  // 3-D maps over [BH][NK][d], 64-row boxes, 128B swizzle
+  const __nv_bfloat16* Q1;  // [BH][NQ][d1], read row by row into TMEM
+  const __nv_bfloat16* Q2;  // [BH][NQ][d2]
   float* L;
   float* LSE1;
   float* LSE2;

@@ -295,10 +295,10 @@ streamkl_status prepare_fwd(const streamkl_problem* prob, const void* Q1, const 
   DeviceInfo* dev = nullptr;
   if ((st = current_device(&dev)) != STREAMKL_OK) return st;
   const int64_t BH = static_cast<int64_t>(prob->B) * prob->H;
-  if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, skl::kFwdBQ, &p->tmQ1)) != STREAMKL_OK) return st;
   if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kFwdBK, &p->tmK1)) != STREAMKL_OK) return st;
-  if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, skl::kFwdBQ, &p->tmQ2)) != STREAMKL_OK) return st;
   if ((st = tensor_map(K2, BH, prob->NK, prob->d2, skl::kFwdBK, &p->tmK2)) != STREAMKL_OK) return st;
+  p->Q1 = static_cast<const __nv_bfloat16*>(Q1);
+  p->Q2 = static_cast<const __nv_bfloat16*>(Q2);
   p->L = L;
   p->LSE1 = LSE1;
   p->LSE2 = LSE2;
