@@ -92,6 +92,32 @@ def workload_desc(w: Workload, phase: str) -> dict:
     }
 
 
+def kernel_sources_sha1() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    csrc = ROOT / "attention_kl_distillation_b200" / "csrc"
+    for f in sorted(csrc.iterdir()):
+        if f.suffix in (".cu", ".cuh", ".h"):
+            h.update(f.name.encode())
+            h.update(f.read_bytes())
+    return h.hexdigest()
+
+
+def profiled_traffic(profile: str):
+    """DRAM bytes per full launch recorded in profiles/<profile>, or None when the kernel
+    sources changed since that ncu capture."""
+    import re
+    f = ROOT / "profiles" / profile
+    if not f.exists():
+        return None
+    text = f.read_text()
+    m1 = re.search(r"source-sha1: ([0-9a-f]{40})", text)
+    m2 = re.search(r"dram-bytes-per-full-launch: (\d+)", text)
+    if not (m1 and m2) or m1.group(1) != kernel_sources_sha1():
+        return None
+    return int(m2.group(1))
+
+
 def step_flops(w: Workload, phase: str) -> int:
     return w.fwd_flops() + (w.bwd_flops() if phase == "fwdbwd" else 0)
 
@@ -305,14 +331,18 @@ def main(argv=None):
     peak, hbm, src = peaks()
     fwd_tf = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
     bwd_tf = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if bwd_ms > 0 else None
+    full_size = w == WORKLOADS[args.workload] and args.need == "1111"
+    algo = binding.bwd_algorithm_for(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal)
     if phase == "fwdbwd" and bwd_ms >= fwd_ms:
-        dom = {"kernel": "streamkl_bwd (prep + main + dQ convert kernels)", "achieved": bwd_tf,
-               "flops_per_launch": w.bwd_flops(), "ms": bwd_ms}
+        dom = {"kernel": f"streamkl_bwd, {algo} (prep + main + convert kernels)",
+               "achieved": bwd_tf, "flops_per_launch": w.bwd_flops(), "ms": bwd_ms,
+               "traffic": profiled_traffic(f"bwd_{algo}_kernel_{w.name}_h8.md") if full_size else None}
     else:
         dom = {"kernel": "streamkl_fwd_kernel", "achieved": fwd_tf,
-               "flops_per_launch": w.fwd_flops(), "ms": fwd_ms}
+               "flops_per_launch": w.fwd_flops(), "ms": fwd_ms,
+               "traffic": profiled_traffic(f"fwd_kernel_{w.name}_h8.md") if full_size else None}
     roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": peak, "unit": UNIT,
-                "frac": dom["achieved"] / peak, "traffic": None, "kernel": dom["kernel"],
+                "frac": dom["achieved"] / peak, "traffic": dom["traffic"], "kernel": dom["kernel"],
                 "flops_per_launch": dom["flops_per_launch"], "ms_per_launch": dom["ms"],
                 "peak_source": f"{src} dense bf16 (burst)"}
 
