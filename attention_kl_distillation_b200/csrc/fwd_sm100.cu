@@ -6,33 +6,34 @@
 // Key tiles past the causal frontier are never loaded or multiplied.
 //
 // B200 mapping (one CTA per SM, persistent):
-//   work unit   (bh, 256-row query block) = two 128-row tiles A and B that
-//               share every key tile, so each K tile is read once per 256 rows
-//   warp 0      TMA producer: K1/K2 tiles into a ring of up to six stages
-//               (128-byte swizzle, no multicast)
-//   warp 1      TMEM owner and UMMA issuer: per key tile and query tile,
-//               S1 = Q1 K1^T and S2 = Q2 K2^T (tcgen05.mma kind::f16, fp32
-//               accumulators).  Q lives in TMEM as the A operand, K in shared
-//               memory as B; keeping Q out of shared memory is what leaves room
-//               for a ring deep enough to cover the TMA latency.
-//   warps 2..17 four reduction warpgroups, two per query tile, each owning 32
-//               of the 64 keys of every key tile: thread r owns query row r
-//               (TMEM lane r).  At the start of a unit it copies its row of Q1
-//               (first warpgroup) or Q2 (second) from global memory into TMEM;
-//               per key tile it loads its 32 + 32 logits with tcgen05.ld, frees
-//               the slot and applies the online update in registers (exp2 on
-//               the MUFU pipe, the softmax scale folded into the exponent
-//               argument, packed f32x2 arithmetic elsewhere).  The two key halves
-//               of a row keep separate running states and merge at the end of the
-//               unit.  Four reduction warps per SM sub-partition hide each
-//               other's latencies.
+//   work unit   (bh, 128-row query tile)
+//   warp 0      TMA producer: 128-key tiles of K1/K2 into a ring of up to six
+//               stages (128-byte swizzle, no multicast)
+//   warp 1      TMEM owner and UMMA issuer: per key tile S1 = Q1 K1^T and
+//               S2 = Q2 K2^T (tcgen05.mma kind::f16, M = 128 rows, N = 128
+//               keys, fp32 accumulators).  Q lives in TMEM as the A operand,
+//               K in shared memory as B.  The S products rotate through three
+//               TMEM slots: S1 of the next key tile is queued behind S2 of this
+//               one while the reduction warps read this one, so the tensor
+//               pipe does not drain between key tiles.
+//   warps 2..17 four reduction warpgroups, each owning 32 of the 128 keys of
+//               every key tile: thread r owns query row r (TMEM lane r).  At
+//               the start of a unit they copy the unit's rows of Q1 and Q2 from
+//               global memory into TMEM; per key tile each thread loads its
+//               32 + 32 logits with tcgen05.ld, frees the slots and applies the
+//               online update in registers (exp2 on the MUFU pipe, the softmax
+//               scale folded into the exponent argument, packed f32x2
+//               arithmetic elsewhere).  The four key parts of a row keep
+//               separate running states and merge at the end of the unit.
+//               Four reduction warps per SM sub-partition hide each other's
+//               latencies.
 // The accumulator acc is one fp32 per row: there is no PV product and no
-// output tile.  TMEM: S1/S2 of tile A [0,128), of tile B [128,256); Q1/Q2 of
-// tile A and tile B as bf16 A operands [256, 256 + d1 + d2).
+// output tile.  TMEM: S slots [0,128) [128,256) [256,384); Q1/Q2 as bf16 A
+// operands [384, 384 + (d1 + d2)/2).
 //
-// Units are visited longest first (the last query blocks of a causal problem
+// Units are visited longest first (the last query tiles of a causal problem
 // see the most keys) and dealt to CTAs in a snake order, an approximation of
-// longest-processing-time scheduling; units of one query block across heads
+// longest-processing-time scheduling; units of one query tile across heads
 // run together, so they stream the same key range through L2.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -43,11 +44,11 @@ namespace skl {
 namespace {
 
 constexpr int BQ = kFwdBQ;
-constexpr int NT = kFwdTiles;
 constexpr int BK = kFwdBK;
-constexpr int NH = 2;    // reduction warpgroups per query tile, each owning BK/NH keys of a tile
+constexpr int NH = 4;        // reduction warpgroups, each owning KH keys of every key tile
 constexpr int KH = BK / NH;
-constexpr int NTHREADS = 64 + NT * NH * 128;
+constexpr int NSLOT = 3;     // TMEM slots the S products rotate through
+constexpr int NTHREADS = 64 + NH * 128;
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D1, int D2>
@@ -55,15 +56,15 @@ struct FwdLayout {
   static constexpr int k1_bytes = BK * D1 * 2;
   static constexpr int k2_bytes = BK * D2 * 2;
   static constexpr int stage_bytes = k1_bytes + k2_bytes;
-  static constexpr int handover_bytes = NT * 5 * BQ * 4;
+  static constexpr int handover_bytes = (NH - 1) * 5 * BQ * 4;
   static constexpr int ks_fit = (232448 - 1024 - 512 - handover_bytes) / stage_bytes;
   static constexpr int KSTAGES = ks_fit > 6 ? 6 : ks_fit;
   static constexpr int k_off = 0;
   static constexpr int bar_off = k_off + KSTAGES * stage_bytes;
-  // barriers: qready[NT], qfree[NT], kfull[KS], kempty[KS], sfull[NT], sempty[NT], drain
-  static constexpr int nbar = 1 + 2 * KSTAGES + 4 * NT;
+  // barriers: qready, qfree, kfull[KS][2], kempty[KS][2], sfull[NSLOT], sempty[NSLOT], drain
+  static constexpr int nbar = 3 + 4 * KSTAGES + 2 * NSLOT;
   static constexpr int misc_off = bar_off + nbar * 8;
-  static constexpr int part_off = misc_off + 16;  // key-half partial states [NT][5][BQ] fp32
+  static constexpr int part_off = misc_off + 16;  // key-part states [NH-1][5][BQ] fp32
   static constexpr int total = part_off + handover_bytes;
   static constexpr int alloc = total + 1024;  // slack to align the base to 1024 B
   static_assert(KSTAGES >= 3, "key ring too shallow");
@@ -71,9 +72,24 @@ struct FwdLayout {
   static_assert(k1_bytes % 1024 == 0 && k2_bytes % 1024 == 0,
                 "tiles must keep 1024-byte alignment for the 128B swizzle atoms");
   // TMEM columns
-  __host__ __device__ static constexpr uint32_t s_col(int t) { return t * 2 * BK; }          // S1; S2 at +BK
-  __host__ __device__ static constexpr uint32_t q_col(int t) { return NT * 2 * BK + t * (D1 + D2) / 2; }  // Q1; Q2 at +D1/2
-  static_assert(NT * 2 * BK + NT * (D1 + D2) / 2 <= 512, "TMEM budget exceeded");
+  __host__ __device__ static constexpr uint32_t s_col(int slot) { return slot * BK; }
+  static constexpr uint32_t q_col = NSLOT * BK;  // Q1; Q2 at +D1/2
+  static_assert(NSLOT * BK + (D1 + D2) / 2 <= 512, "TMEM budget exceeded");
+};
+
+// Rotation of the S products through the TMEM slots.  Counted over the CTA's
+// whole run, product k (S1 of a key tile, then its S2) uses slot k mod NSLOT;
+// a slot's two barriers complete one phase per use.  The issuer and the
+// reduction warps step their own copies through the same sequence.
+struct SlotRing {
+  int s = 0;
+  uint32_t ph = 0;  // bit i: parity of slot i's current use
+  __device__ __forceinline__ int slot() const { return s; }
+  __device__ __forceinline__ uint32_t parity() const { return (ph >> s) & 1u; }
+  __device__ __forceinline__ void advance() {
+    ph ^= 1u << s;
+    s = (s == NSLOT - 1) ? 0 : s + 1;
+  }
 };
 
 struct Sched {
@@ -94,15 +110,14 @@ struct Sched {
 
 struct Unit {
   int bh, q0;
-  int kt_lo;       // first key tile of this unit (split-K chunk start; 0 without split)
-  int nkt[NT];     // end of the key tiles each query tile processes (<= kt_lo: none)
-  int kt_mask[NT]; // key tiles [kt_mask, nkt) need element masks
-  int nkt_max;
-  int split;       // key split index (0 without split)
+  int kt_lo;    // first key tile of this unit (split-K chunk start; 0 without split)
+  int nkt;      // end of the key tiles the tile processes (<= kt_lo: none)
+  int kt_mask;  // key tiles [kt_mask, nkt) need element masks
+  int split;    // key split index (0 without split)
 };
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
-  const int nqb = (p.NQ + BQ * NT - 1) / (BQ * NT);
+  const int nqb = (p.NQ + BQ - 1) / BQ;
   Unit w;
   w.split = 0;
   if (p.nsplit > 1) {
@@ -110,27 +125,17 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     u /= p.nsplit;
   }
   w.bh = u % p.BH;
-  w.q0 = (nqb - 1 - u / p.BH) * (BQ * NT);  // longest (last) query blocks first
+  w.q0 = (nqb - 1 - u / p.BH) * BQ;  // longest (last) query tiles first
   const int nkt_all = (p.NK + BK - 1) / BK;
-  const int tail = (p.NK % BK) ? nkt_all - 1 : nkt_all;
   const int off = p.NK - p.NQ;
   w.kt_lo = p.nsplit > 1 ? w.split * p.kt_chunk : 0;
   const int kt_hi = p.nsplit > 1 ? min(nkt_all, w.kt_lo + p.kt_chunk) : nkt_all;
-  w.nkt_max = w.kt_lo;
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const int r0 = w.q0 + t * BQ;
-    int nkt = kt_hi, km = tail;
-    if (r0 >= p.NQ) {
-      nkt = 0;
-    } else if (p.causal) {
-      const int last = min(r0 + BQ - 1, p.NQ - 1) + off;  // last key any row of the tile sees
-      nkt = min(kt_hi, last / BK + 1);
-      km = min(km, (r0 + off + 1) / BK);  // first tile the first row cannot fully see
-    }
-    w.nkt[t] = nkt;
-    w.kt_mask[t] = km;
-    w.nkt_max = max(w.nkt_max, nkt);
+  w.nkt = kt_hi;
+  w.kt_mask = (p.NK % BK) ? nkt_all - 1 : nkt_all;
+  if (p.causal) {
+    const int last = min(w.q0 + BQ - 1, p.NQ - 1) + off;  // last key any row of the tile sees
+    w.nkt = min(kt_hi, last / BK + 1);
+    w.kt_mask = min(w.kt_mask, (w.q0 + off + 1) / BK);  // first tile the first row cannot fully see
   }
   return w;
 }
@@ -205,27 +210,33 @@ __device__ __forceinline__ void tile_update(const uint32_t (&a)[KH], const uint3
   st.m2 = m2n;
 }
 
-// Copies query row `row` of Q ([BH][NQ][D] bf16) into TMEM columns [col,
-// col + D/2) of this thread's lane as the A operand of the S products (two
-// features per 32-bit column, the lower feature in the low half); rows past
-// NQ are zero.
-template <int D>
-__device__ __forceinline__ void stage_q_row(const __nv_bfloat16* Q, int bh, int NQ, int row,
+// Copies this thread's query row of Q1 and Q2 ([BH][NQ][d] bf16) into TMEM
+// as the A operands of the S products: two features per 32-bit column, the
+// lower feature in the low half, Q2 after Q1's d1/2 columns.  The rows are
+// copied in chunks of 32 features, chunk g by warpgroup g mod NH, so the four
+// warpgroups share the work.  Rows past NQ are zero.
+template <int D1, int D2>
+__device__ __forceinline__ void stage_q_row(const FwdParams& p, int bh, int row, int part,
                                             uint32_t taddr) {
-  const bool ok = row < NQ;
-  const uint4* src = reinterpret_cast<const uint4*>(Q + (static_cast<size_t>(bh) * NQ + (ok ? row : 0)) * D);
+  const bool ok = row < p.NQ;
+  const size_t r = static_cast<size_t>(bh) * p.NQ + (ok ? row : 0);
+  const uint4* src1 = reinterpret_cast<const uint4*>(p.Q1 + r * D1);
+  const uint4* src2 = reinterpret_cast<const uint4*>(p.Q2 + r * D2);
+  constexpr int C1 = D1 / 32, C = (D1 + D2) / 32;
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {  // 32 features = 16 columns per chunk
+  for (int g = 0; g < C; ++g) {
+    if (g % NH != part) continue;
+    const uint4* src = g < C1 ? src1 + g * 4 : src2 + (g - C1) * 4;
     uint32_t v[16];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      uint4 x = ok ? __ldg(src + c * 4 + k) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 x = ok ? __ldg(src + k) : make_uint4(0u, 0u, 0u, 0u);
       v[4 * k + 0] = x.x;
       v[4 * k + 1] = x.y;
       v[4 * k + 2] = x.z;
       v[4 * k + 3] = x.w;
     }
-    tmem_st_32x32b_x16(taddr + c * 16, v);
+    tmem_st_32x32b_x16(taddr + g * 16, v);  // 32 features = 16 columns
   }
 }
 
@@ -237,13 +248,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off);
-  uint64_t* qready = bars + 0;    // [NT]: the tile's Q rows of this unit are in TMEM
-  uint64_t* qfree = qready + NT;  // [NT]: the UMMAs of the previous unit have read them
-  uint64_t* kfull = qfree + NT;
-  uint64_t* kempty = kfull + KS;
-  uint64_t* sfull = kempty + KS;  // [NT]
-  uint64_t* sempty = sfull + NT;  // [NT]
-  uint64_t* drain = sempty + NT;
+  uint64_t* qready = bars + 0;    // this unit's Q rows are in TMEM
+  uint64_t* qfree = qready + 1;   // the UMMAs of the previous unit have read them
+  // [KS][2]: the K1 and K2 halves of a stage are filled and freed separately,
+  // so K1 of a later key tile is in flight as soon as S1 has read this one
+  uint64_t* kfull = qfree + 1;
+  uint64_t* kempty = kfull + 2 * KS;
+  uint64_t* sfull = kempty + 2 * KS;  // [NSLOT]
+  uint64_t* sempty = sfull + NSLOT;   // [NSLOT]
+  uint64_t* drain = sempty + NSLOT;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::misc_off + 4);
 
@@ -253,17 +266,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    for (int t = 0; t < NT; ++t) {
-      mbar_init(&qready[t], 4 * NH);  // every reduction warp of the tile wrote its Q rows
-      mbar_init(&qfree[t], 1);
-    }
-    for (int s = 0; s < KS; ++s) {
+    mbar_init(qready, 4 * NH);  // every reduction warp wrote its share of the Q rows
+    mbar_init(qfree, 1);
+    for (int s = 0; s < 2 * KS; ++s) {
       mbar_init(&kfull[s], 1);
       mbar_init(&kempty[s], 1);
     }
-    for (int t = 0; t < NT; ++t) {
-      mbar_init(&sfull[t], 1);
-      mbar_init(&sempty[t], 4 * NH);  // one arrival per reduction warp of that tile
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 4 * NH);  // one arrival per reduction warp
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -289,22 +300,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     if (lane == 0) {
       int ks = 0;
       uint32_t kph = 0;
-      uint32_t armed_k[KS] = {};  // last armed phase + 1 (0 = never)
+      uint32_t armed_k[2 * KS] = {};  // last armed phase + 1 (0 = never)
       int u;
       bool ok = true;
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
-        if (w.nkt_max <= w.kt_lo) continue;  // split chunk past every row's frontier
-        for (int kt = w.kt_lo; kt < (p.withhold_keys ? w.kt_lo : w.nkt_max); ++kt) {
-          if (!(ok = mbar_wait(&kempty[ks], kph ^ 1, ctl))) break;
-          mbar_arrive_expect_tx(&kfull[ks], Lay::stage_bytes);
+        if (w.nkt <= w.kt_lo) continue;  // split chunk past every row's frontier
+        for (int kt = w.kt_lo; kt < (p.withhold_keys ? w.kt_lo : w.nkt); ++kt) {
+          if (!(ok = mbar_wait(&kempty[2 * ks], kph ^ 1, ctl))) break;
+          mbar_arrive_expect_tx(&kfull[2 * ks], Lay::k1_bytes);
 #pragma unroll
           for (int b = 0; b < D1 / 64; ++b)
-            tma_load_3d(k1_s(ks) + b * (BK * 128), &p.tmK1, &kfull[ks], b * 64, kt * BK, w.bh);
+            tma_load_3d(k1_s(ks) + b * (BK * 128), &p.tmK1, &kfull[2 * ks], b * 64, kt * BK, w.bh);
+          armed_k[2 * ks] = kph + 1;
+          if (!(ok = mbar_wait(&kempty[2 * ks + 1], kph ^ 1, ctl))) break;
+          mbar_arrive_expect_tx(&kfull[2 * ks + 1], Lay::k2_bytes);
 #pragma unroll
           for (int b = 0; b < D2 / 64; ++b)
-            tma_load_3d(k2_s(ks) + b * (BK * 128), &p.tmK2, &kfull[ks], b * 64, kt * BK, w.bh);
-          armed_k[ks] = kph + 1;
+            tma_load_3d(k2_s(ks) + b * (BK * 128), &p.tmK2, &kfull[2 * ks + 1], b * 64, kt * BK, w.bh);
+          armed_k[2 * ks + 1] = kph + 1;
           if (++ks == KS) {
             ks = 0;
             kph ^= 1;
@@ -315,7 +329,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
         // Aborting: let the copies already in flight land before the CTA exits.
         volatile int zero = 0;
         WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
-        for (int s = 0; s < KS; ++s)
+        for (int s = 0; s < 2 * KS; ++s)
           if (armed_k[s]) mbar_wait(&kfull[s], armed_k[s] - 1, dctl);
       }
     }
@@ -323,55 +337,59 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(BQ, BK);
+      const uint32_t a1 = tmem_base + Lay::q_col, a2 = a1 + D1 / 2;
       int ks = 0;
       uint32_t kph = 0, qph = 0;
-      uint32_t sph[NT] = {};
+      SlotRing ring;
       int u;
       bool ok = true;
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
-        if (w.nkt_max <= w.kt_lo) continue;
-#pragma unroll
-        for (int t = 0; t < NT; ++t)  // Q of this unit is in TMEM
-          if (ok) ok = mbar_wait(&qready[t], qph, ctl);
-        if (!ok) break;
+        if (w.nkt <= w.kt_lo) continue;
+        if (!(ok = mbar_wait(qready, qph, ctl))) break;  // Q of this unit is in TMEM
         qph ^= 1;
         tc_fence_after();
-        for (int kt = w.kt_lo; kt < w.nkt_max && ok; ++kt) {
-          if (!(ok = mbar_wait(&kfull[ks], kph, ctl))) break;
+        for (int kt = w.kt_lo; kt < w.nkt; ++kt) {
           // Descriptors built once per stage; each UMMA below costs an add and the
           // MMA itself, so this thread keeps up although it shares its SM
           // sub-partition with four busy reduction warps.
           const uint64_t b1 = sdesc_sw128(smem_u32(k1_s(ks)), 16, 1024);
           const uint64_t b2 = sdesc_sw128(smem_u32(k2_s(ks)), 16, 1024);
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            if (kt >= w.nkt[t]) continue;
-            if (!(ok = mbar_wait(&sempty[t], sph[t] ^ 1, ctl))) break;
-            sph[t] ^= 1;
-            tc_fence_after();
-            const uint32_t d1 = tmem_base + Lay::s_col(t), d2 = d1 + BK;
-            const uint32_t a1 = tmem_base + Lay::q_col(t), a2 = a1 + D1 / 2;
+          // S1 into the next slot once K1 has landed and the reduction warps
+          // have read the slot out
+          if (!(ok = mbar_wait(&kfull[2 * ks], kph, ctl))) break;
+          if (!(ok = mbar_wait(&sempty[ring.slot()], ring.parity() ^ 1, ctl))) break;
+          tc_fence_after();
+          {
+            const uint32_t d = tmem_base + Lay::s_col(ring.slot());
 #pragma unroll
             for (int kk = 0; kk < D1 / 16; ++kk)
-              umma_bf16_ts(d1, a1 + kk * 8,
+              umma_bf16_ts(d, a1 + kk * 8,
                            sdesc_advance(b1, (kk >> 2) * (BK * 128) + (kk & 3) * 32), idesc, kk > 0);
+            umma_commit(&sfull[ring.slot()]);
+            umma_commit(&kempty[2 * ks]);
+            ring.advance();
+          }
+          if (!(ok = mbar_wait(&kfull[2 * ks + 1], kph, ctl))) break;
+          if (!(ok = mbar_wait(&sempty[ring.slot()], ring.parity() ^ 1, ctl))) break;
+          tc_fence_after();
+          {
+            const uint32_t d = tmem_base + Lay::s_col(ring.slot());
 #pragma unroll
             for (int kk = 0; kk < D2 / 16; ++kk)
-              umma_bf16_ts(d2, a2 + kk * 8,
+              umma_bf16_ts(d, a2 + kk * 8,
                            sdesc_advance(b2, (kk >> 2) * (BK * 128) + (kk & 3) * 32), idesc, kk > 0);
-            umma_commit(&sfull[t]);
+            umma_commit(&sfull[ring.slot()]);
+            umma_commit(&kempty[2 * ks + 1]);
+            ring.advance();
           }
-          if (!ok) break;
-          umma_commit(&kempty[ks]);
           if (++ks == KS) {
             ks = 0;
             kph ^= 1;
           }
         }
         if (!ok) break;
-#pragma unroll
-        for (int t = 0; t < NT; ++t) umma_commit(&qfree[t]);  // once this unit's UMMAs are done
+        umma_commit(qfree);  // once this unit's UMMAs are done
       }
       // Every UMMA issued by this thread completes before TMEM is released.
       umma_commit(drain);
@@ -381,79 +399,90 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     }
   } else {
     // ------------------------------------------------------------ reduction
-    const int rw = (warp - 2) >> 2;
-    const int t = rw / NH;   // query tile of this warpgroup
-    const int hf = rw % NH;  // which KH keys of every key tile it owns
+    const int hf = (warp - 2) >> 2;  // which KH keys of every key tile this warpgroup owns
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t tlane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    float* part = reinterpret_cast<float*>(smem + Lay::part_off) + t * 5 * BQ;
+    float* part = reinterpret_cast<float*>(smem + Lay::part_off);
     const int off = p.NK - p.NQ;
-    uint32_t sph = 0, qfph = 0;
+    uint32_t qfph = 0;
+    SlotRing ring;
     int u;
     bool ok = true;
     while (ok && sched.next(u)) {
       const Unit w = decode_unit(p, u);
-      if (w.nkt_max <= w.kt_lo) continue;
-      const int i_abs = w.q0 + t * BQ + row;
+      if (w.nkt <= w.kt_lo) continue;
+      const int i_abs = w.q0 + row;
       // This unit's Q rows into TMEM, once the previous unit's UMMAs have read them.
-      if (!(ok = mbar_wait(&qfree[t], qfph ^ 1, ctl))) break;
+      if (!(ok = mbar_wait(qfree, qfph ^ 1, ctl))) break;
       qfph ^= 1;
       tc_fence_after();
-      if (hf == 0)
-        stage_q_row<D1>(p.Q1, w.bh, p.NQ, i_abs, tlane + Lay::q_col(t));
-      else
-        stage_q_row<D2>(p.Q2, w.bh, p.NQ, i_abs, tlane + Lay::q_col(t) + D1 / 2);
+      stage_q_row<D1, D2>(p, w.bh, i_abs, hf, tlane + Lay::q_col);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&qready[t]);
+      if (lane == 0) mbar_arrive(qready);
       const int lim = p.causal ? min(p.NK, i_abs + off + 1) : p.NK;  // visible keys [0, lim)
       RowState st{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
-      const int nkt = w.nkt[t];
-      for (int kt = w.kt_lo; kt < nkt; ++kt) {
-        if (!(ok = mbar_wait(&sfull[t], sph, ctl))) break;
-        sph ^= 1;
-        tc_fence_after();
+      for (int kt = w.kt_lo; kt < w.nkt; ++kt) {
         uint32_t a[KH], b[KH];
-        const uint32_t tcol = tlane + Lay::s_col(t) + hf * KH;
-        tmem_ld_32x32b<KH>(tcol, a);
-        tmem_ld_32x32b<KH>(tcol + BK, b);
+        const int sa = ring.slot();
+        if (!(ok = mbar_wait(&sfull[sa], ring.parity(), ctl))) break;
+        ring.advance();
+        tc_fence_after();
+        tmem_ld_32x32b<KH>(tlane + Lay::s_col(sa) + hf * KH, a);
+        const int sb = ring.slot();
+        if (!(ok = mbar_wait(&sfull[sb], ring.parity(), ctl))) break;
+        ring.advance();
+        tc_fence_after();
+        tmem_ld_32x32b<KH>(tlane + Lay::s_col(sb) + hf * KH, b);
         tmem_ld_wait();
         reg_fence(a);
         reg_fence(b);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sempty[t]);
-        if (kt >= w.kt_mask[t])
+        if (lane == 0) {
+          mbar_arrive(&sempty[sa]);
+          mbar_arrive(&sempty[sb]);
+        }
+        if (kt >= w.kt_mask)
           tile_update<true>(a, b, p.c1, p.c2, lim - kt * BK - hf * KH, st);
         else
           tile_update<false>(a, b, p.c1, p.c2, KH, st);
       }
       if (!ok) break;
-      // Merge the key halves of every row (same rescaling as the split-K merge):
-      // the second warpgroup hands its state over through shared memory.
-      if (hf == 1) {
-        part[0 * BQ + row] = st.m1;
-        part[1 * BQ + row] = st.m2;
-        part[2 * BQ + row] = st.l1;
-        part[3 * BQ + row] = st.l2;
-        part[4 * BQ + row] = st.acc;
+      // Merge the key parts of every row (same rescaling as the split-K merge):
+      // the other warpgroups hand their states over through shared memory.
+      if (hf > 0) {
+        float* slot = part + (hf - 1) * 5 * BQ;
+        slot[0 * BQ + row] = st.m1;
+        slot[1 * BQ + row] = st.m2;
+        slot[2 * BQ + row] = st.l1;
+        slot[3 * BQ + row] = st.l2;
+        slot[4 * BQ + row] = st.acc;
       }
-      named_bar_sync(1 + t, NH * 128);
+      named_bar_sync(1, NH * 128);
       if (hf == 0) {
-        const float om1 = part[0 * BQ + row], om2 = part[1 * BQ + row];
-        const float m1 = fmaxf(st.m1, om1), m2 = fmaxf(st.m2, om2);
-        const float fa1 = ex2(st.m1 - m1), fb1 = ex2(om1 - m1);  // 0 for a half with no key
-        const float fa2 = ex2(st.m2 - m2), fb2 = ex2(om2 - m2);
-        st.l1 = fmaf(st.l1, fa1, part[2 * BQ + row] * fb1);
-        st.l2 = fmaf(st.l2, fa2, part[3 * BQ + row] * fb2);
-        st.acc = fmaf(st.acc, fa1, part[4 * BQ + row] * fb1);
-        st.m1 = m1;
-        st.m2 = m2;
+#pragma unroll
+        for (int o = 0; o < NH - 1; ++o) {
+          const float* slot = part + o * 5 * BQ;
+          const float om1 = slot[0 * BQ + row], om2 = slot[1 * BQ + row];
+          const float m1 = fmaxf(st.m1, om1), m2 = fmaxf(st.m2, om2);
+          // a part with no visible key has m = -inf and weight 0; two such
+          // parts keep the empty state
+          const float fa1 = st.m1 == -INFINITY ? 0.f : ex2(st.m1 - m1);
+          const float fb1 = om1 == -INFINITY ? 0.f : ex2(om1 - m1);
+          const float fa2 = st.m2 == -INFINITY ? 0.f : ex2(st.m2 - m2);
+          const float fb2 = om2 == -INFINITY ? 0.f : ex2(om2 - m2);
+          st.l1 = fmaf(st.l1, fa1, slot[2 * BQ + row] * fb1);
+          st.l2 = fmaf(st.l2, fa2, slot[3 * BQ + row] * fb2);
+          st.acc = fmaf(st.acc, fa1, slot[4 * BQ + row] * fb1);
+          st.m1 = m1;
+          st.m2 = m2;
+        }
       }
-      named_bar_sync(1 + t, NH * 128);  // the handover slot may be reused
-      if (hf == 0 && i_abs < p.NQ && w.q0 + t * BQ < p.NQ) {
+      named_bar_sync(1, NH * 128);  // the handover slots may be reused
+      if (hf == 0 && i_abs < p.NQ) {
         const size_t o = static_cast<size_t>(w.bh) * p.NQ + i_abs;
         if (p.nsplit > 1) {
           // partial state of this key chunk, merged by streamkl_fwd_merge_kernel
@@ -464,7 +493,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
           dst[2 * rows] = st.l1;
           dst[3 * rows] = st.l2;
           dst[4 * rows] = st.acc;
-        } else if (nkt > 0) {
+        } else {
           const float lg1 = lg2(st.l1), lg2v = lg2(st.l2);
           p.LSE1[o] = kLn2 * (st.m1 + lg1);
           p.LSE2[o] = kLn2 * (st.m2 + lg2v);

@@ -9,15 +9,14 @@
 
 namespace skl {
 
-// Rows of Q in one forward tile (the UMMA M dimension and the TMEM lanes);
-// a work unit holds kFwdTiles such tiles that share every key tile.
+// Rows of Q in one forward tile and work unit (the UMMA M dimension and the
+// TMEM lanes).
 constexpr int kFwdBQ = 128;
-constexpr int kFwdTiles = 2;
 // Keys per forward tile (UMMA N).
-constexpr int kFwdBK = 64;
+constexpr int kFwdBK = 128;
 
 struct FwdParams {
-  CUtensorMap tmK1, tmK2;  // 3-D maps over [BH][NK][d], 64-row boxes, 128B swizzle
+  CUtensorMap tmK1, tmK2;  // 3-D maps over [BH][NK][d], 128-row boxes, 128B swizzle
   const __nv_bfloat16* Q1;  // [BH][NQ][d1], read row by row into TMEM
   const __nv_bfloat16* Q2;  // [BH][NQ][d2]
   float* L;
@@ -120,9 +119,9 @@ cudaError_t launch_bwd_convert(const BwdConvertParams& p, int num_sms, cudaStrea
 
 __host__ __device__ inline int bwd_units(int BH, int NK) { return BH * ((NK + kBwdBK - 1) / kBwdBK); }
 
-// Work units of the forward: (bh, 256-row query block) pairs, times the key splits.
+// Work units of the forward: (bh, 128-row query tile) pairs, times the key splits.
 __host__ __device__ inline int fwd_units(int BH, int NQ, int nsplit = 1) {
-  return BH * ((NQ + kFwdBQ * kFwdTiles - 1) / (kFwdBQ * kFwdTiles)) * (nsplit > 1 ? nsplit : 1);
+  return BH * ((NQ + kFwdBQ - 1) / kFwdBQ) * (nsplit > 1 ? nsplit : 1);
 }
 
 }  // namespace skl

@@ -82,8 +82,8 @@ streamkl_status streamkl_fwd(const streamkl_problem *prob, const void *Q1, const
  * Split-K forward (section 3, "Variante Split-K": for few query rows, e.g. a
  * decode step with N_Q = 1, the keys are partitioned across thread blocks so
  * that every SM has work).  Same results as streamkl_fwd within rounding.
- * The keys of every 256-row query block are cut into `nsplit` chunks of equal
- * length (in 64-key tiles); each chunk's blocks write partial row states
+ * The keys of every 128-row query tile are cut into `nsplit` chunks of equal
+ * length (in 128-key tiles); each chunk's tiles write partial row states
  * (m1, m2, l1, l2, acc) to `workspace`, and a merge kernel combines them into
  * L, LSE1, LSE2.  nsplit >= 1 (1 = no split); nsplit above the number of key
  * tiles is clamped.  workspace: streamkl_fwd_splitk_workspace_size(prob,

@@ -128,8 +128,8 @@ def test_bwd_algorithm_selection():
 def test_splitk_workspace_and_validation():
     assert B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 3) >= 3 * 5 * 2 * 10 * 4
     assert B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 0) == 0
-    # nsplit beyond the 10 key tiles is clamped
-    assert B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 50) == B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 10)
+    # nsplit beyond the 5 key tiles of 128 is clamped
+    assert B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 50) == B.splitk_workspace_size(1, 2, 10, 640, 64, 64, 5)
     lib = B.lib()
     prob = B.problem(1, 2, 10, 640, 64, 64)
     v = ctypes.c_void_p
