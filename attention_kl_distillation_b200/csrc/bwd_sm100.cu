@@ -33,6 +33,15 @@
 //               of a unit converts the dK accumulators to bf16 and stores them.
 // TMEM (512 columns): S1^T [0,64) S2^T [64,128) dK1 [128,128+d1) dK2 [..,+d2)
 //                     dQ1^T [384,448) dQ2^T [448,512).
+//
+// Gradient sets (the page's two configurations, same section): the kernel is
+// instantiated for SEL = 1 (teacher side only: dQ1, dK1 -- Configuration 2,
+// P2 fixed), SEL = 2 (student side only: dQ2, dK2 -- Configuration 1, P1
+// fixed, standard distillation) and SEL = 3 (both).  A one-sided instance
+// forms, stores and contracts only its own dS, keeps a dQ accumulator of that
+// side's width only, and for SEL = 1 skips the P2 exponential (dS1 needs the
+// student only through its log-probability, which is linear in S2).  Both S
+// products are recomputed in every configuration.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -52,8 +61,8 @@ constexpr int NTHREADS = (DQ_WARP0 + 4) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kColS1 = 0, kColS2 = 64, kColDK1 = 128, kColDQ1 = 384, kColDQ2 = 448;
 
-template <int D1, int D2>
-struct BwdLayout {
+template <int D1, int D2, int NDT>
+struct BwdLayout {  // NDT: dS tiles per buffer (1 or 2 gradient sides)
   static constexpr int k1_bytes = BK * D1 * 2;
   static constexpr int k2_bytes = BK * D2 * 2;
   static constexpr int q1_bytes = BQ * D1 * 2;
@@ -65,7 +74,7 @@ struct BwdLayout {
   // must be in flight while step t is contracted.
   static constexpr int fixed_bytes = k1_bytes + k2_bytes + 1024 + 512;
   static constexpr bool fits(int q, int d) {
-    return fixed_bytes + q * qstage_bytes + d * 2 * ds_bytes <= 232448;
+    return fixed_bytes + q * qstage_bytes + d * NDT * ds_bytes <= 232448;
   }
   static constexpr int QSTAGES = fits(4, 2) ? 4 : (fits(3, 2) ? 3 : (fits(4, 1) ? 4 : 3));
   static constexpr int DSBUF = fits(QSTAGES, 2) ? 2 : 1;
@@ -73,7 +82,7 @@ struct BwdLayout {
   static constexpr int k2_off = k1_off + k1_bytes;
   static constexpr int q_off = k2_off + k2_bytes;
   static constexpr int ds_off = q_off + QSTAGES * qstage_bytes;
-  static constexpr int bar_off = ds_off + DSBUF * 2 * ds_bytes;
+  static constexpr int bar_off = ds_off + DSBUF * NDT * ds_bytes;
   // kfull kempty qfull[Q] qempty[Q] sfull sempty dsfull[D] dsempty[D] dqfull dqempty1
   // dqempty2 dkfull dkempty ufull[2] uempty[2] drain
   static constexpr int nbar = 2 + 2 * QSTAGES + 2 + 2 * DSBUF + 5 + 4 + 1;
@@ -135,7 +144,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 //   dS1 = s1 dL P1 (ln2 (u1 - u2) - L),   dS2 = s2 dL (P2 - P1)
 // MASK: visible iff key < NK and (not causal or q >= thr), with thr the first
 // visible query index of this half for this key.
-template <bool MASK>
+template <bool MASK, bool G1, bool G2>
 __device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_t (&s2)[QPW],
                                         const float* rr, float c1, float c2, bool key_ok, int thr,
                                         uint32_t (&w1)[QPW / 2], uint32_t (&w2)[QPW / 2]) {
@@ -149,8 +158,8 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_
       const float4 nb1 = *reinterpret_cast<const float4*>(rr + 0 * BQ + q);
       const float4 nb2 = *reinterpret_cast<const float4*>(rr + 1 * BQ + q);
       const float4 nL = *reinterpret_cast<const float4*>(rr + 2 * BQ + q);
-      const float4 g1 = *reinterpret_cast<const float4*>(rr + 3 * BQ + q);
-      const float4 g2 = *reinterpret_cast<const float4*>(rr + 4 * BQ + q);
+      const float4 g1 = G1 ? *reinterpret_cast<const float4*>(rr + 3 * BQ + q) : float4{};
+      const float4 g2 = G2 ? *reinterpret_cast<const float4*>(rr + 4 * BQ + q) : float4{};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {  // a pair of queries
         const int i = q + 2 * e;
@@ -159,15 +168,20 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_
         const float2 B1 = e ? make_float2(nb1.z, nb1.w) : make_float2(nb1.x, nb1.y);
         const float2 B2 = e ? make_float2(nb2.z, nb2.w) : make_float2(nb2.x, nb2.y);
         const float2 NL = e ? make_float2(nL.z, nL.w) : make_float2(nL.x, nL.y);
-        const float2 G1 = e ? make_float2(g1.z, g1.w) : make_float2(g1.x, g1.y);
-        const float2 G2 = e ? make_float2(g2.z, g2.w) : make_float2(g2.x, g2.y);
+        const float2 Gs1 = e ? make_float2(g1.z, g1.w) : make_float2(g1.x, g1.y);
+        const float2 Gs2 = e ? make_float2(g2.z, g2.w) : make_float2(g2.x, g2.y);
         const float2 u1 = __ffma2_rn(S1, C1, B1);
         const float2 u2 = __ffma2_rn(S2, C2, B2);
         const float2 P1 = make_float2(ex2(u1.x), ex2(u1.y));
-        const float2 P2 = make_float2(ex2(u2.x), ex2(u2.y));
-        const float2 t = __ffma2_rn(__ffma2_rn(u2, NEG1, u1), LN2, NL);
-        float2 d1 = __fmul2_rn(__fmul2_rn(P1, t), G1);
-        float2 d2 = __fmul2_rn(__ffma2_rn(P1, NEG1, P2), G2);
+        float2 d1 = make_float2(0.f, 0.f), d2 = make_float2(0.f, 0.f);
+        if (G1) {
+          const float2 t = __ffma2_rn(__ffma2_rn(u2, NEG1, u1), LN2, NL);
+          d1 = __fmul2_rn(__fmul2_rn(P1, t), Gs1);
+        }
+        if (G2) {
+          const float2 P2 = make_float2(ex2(u2.x), ex2(u2.y));
+          d2 = __fmul2_rn(__ffma2_rn(P1, NEG1, P2), Gs2);
+        }
         if (MASK) {
           const bool vx = key_ok && i >= thr, vy = key_ok && i + 1 >= thr;
           d1.x = vx ? d1.x : 0.f;
@@ -175,8 +189,8 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_
           d1.y = vy ? d1.y : 0.f;
           d2.y = vy ? d2.y : 0.f;
         }
-        w1[c * 4 + h * 2 + e] = pack_bf16(d1.x, d1.y);
-        w2[c * 4 + h * 2 + e] = pack_bf16(d2.x, d2.y);
+        if (G1) w1[c * 4 + h * 2 + e] = pack_bf16(d1.x, d1.y);
+        if (G2) w2[c * 4 + h * 2 + e] = pack_bf16(d2.x, d2.y);
       }
     }
   }
@@ -184,14 +198,15 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_
 
 // Stores the packed dS row segments of one key into the 128B-swizzled tiles:
 // 16-byte chunk c0 + c of row j lands at chunk (c0 + c) ^ (j mod 8).
+template <bool G1, bool G2>
 __device__ __forceinline__ void store_ds(const uint32_t (&w1)[QPW / 2],
                                          const uint32_t (&w2)[QPW / 2], int j, int c0,
                                          uint32_t ds1_row, uint32_t ds2_row) {
 #pragma unroll
   for (int c = 0; c < QPW / 8; ++c) {
     const uint32_t sw = static_cast<uint32_t>(((c0 + c) ^ (j & 7)) << 4);
-    st_shared_v4(ds1_row + sw, w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
-    st_shared_v4(ds2_row + sw, w2[4 * c], w2[4 * c + 1], w2[4 * c + 2], w2[4 * c + 3]);
+    if (G1) st_shared_v4(ds1_row + sw, w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
+    if (G2) st_shared_v4(ds2_row + sw, w2[4 * c], w2[4 * c + 1], w2[4 * c + 2], w2[4 * c + 3]);
   }
 }
 
@@ -204,12 +219,15 @@ __device__ __forceinline__ void red_dq(float* base, const uint32_t (&v)[32], int
     if (FULL || i < nvalid) atomicAdd(base + i * LDQ, __uint_as_float(v[i]));
 }
 
-template <int D1, int D2>
+template <int D1, int D2, int SEL>
 __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_constant__ BwdParams p) {
-  using Lay = BwdLayout<D1, D2>;
+  constexpr bool G1 = (SEL & 1) != 0, G2 = (SEL & 2) != 0;
+  using Lay = BwdLayout<D1, D2, (G1 ? 1 : 0) + (G2 ? 1 : 0)>;
   constexpr int QST = Lay::QSTAGES;
   constexpr int DSB = Lay::DSBUF;
-  constexpr int LDQ = D1 + D2;
+  // dQ accumulator row: the wanted sides only, teacher first
+  constexpr int LDQ = (G1 ? D1 : 0) + (G2 ? D2 : 0);
+  constexpr int DQ2_COL = G1 ? D1 : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -288,8 +306,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
     return reinterpret_cast<float*>(smem + Lay::q_off + s * Lay::qstage_bytes + Lay::q1_bytes +
                                     Lay::q2_bytes);
   };
-  auto ds1_s = [&](int b) { return smem + Lay::ds_off + b * 2 * Lay::ds_bytes; };
-  auto ds2_s = [&](int b) { return smem + Lay::ds_off + b * 2 * Lay::ds_bytes + Lay::ds_bytes; };
+  constexpr int NDT = (G1 ? 1 : 0) + (G2 ? 1 : 0);
+  auto ds1_s = [&](int b) { return smem + Lay::ds_off + b * NDT * Lay::ds_bytes; };
+  auto ds2_s = [&](int b) {
+    return smem + Lay::ds_off + b * NDT * Lay::ds_bytes + (G1 ? Lay::ds_bytes : 0);
+  };
   const int off = p.NK - p.NQ;
 
   if (warp == 0) {
@@ -426,32 +447,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           // B = Q_t read MN-major (features contiguous; 64-feature chunks 8 KB apart).
 #pragma unroll
           for (int kk = 0; kk < BQ / 16; ++kk) {
-            if (p.want_dk1)
+            if (G1 && p.want_dk1)
               umma_bf16_ss(tmem_base + kColDK1, sdesc_sw128(smem_u32(ds1_s(db)) + kk * 32, 16, 1024),
                            sdesc_sw128(smem_u32(q1_s(qs_r)) + kk * 2048, BQ * 128, 1024), idK1, (t > 0 || kk > 0));
-            if (p.want_dk2)
+            if (G2 && p.want_dk2)
               umma_bf16_ss(tmem_base + kColDK1 + D1, sdesc_sw128(smem_u32(ds2_s(db)) + kk * 32, 16, 1024),
                            sdesc_sw128(smem_u32(q2_s(qs_r)) + kk * 2048, BQ * 128, 1024), idK2, (t > 0 || kk > 0));
           }
           // dQ_t^T = K_t^T (s_t dS_t)^T : A = K tile read MN-major (64-feature chunks
           // 16 KB apart), B = dS^T read MN-major (64 queries contiguous per key).
-          if (!(ok = mbar_wait(&dqempty[0], dqph[0] ^ 1, ctl))) break;
-          dqph[0] ^= 1;
-          tc_fence_after();
-          if (p.want_dq1) {
+          if (G1) {
+            if (!(ok = mbar_wait(&dqempty[0], dqph[0] ^ 1, ctl))) break;
+            dqph[0] ^= 1;
+            tc_fence_after();
+            if (p.want_dq1) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma_bf16_ss(tmem_base + kColDQ1, sdesc_advance(k1m, kk * 2048),
-                           sdesc_advance(d1m, kk * 2048), idQ1, kk > 0);
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma_bf16_ss(tmem_base + kColDQ1, sdesc_advance(k1m, kk * 2048),
+                             sdesc_advance(d1m, kk * 2048), idQ1, kk > 0);
+            }
           }
-          if (!(ok = mbar_wait(&dqempty[1], dqph[1] ^ 1, ctl))) break;
-          dqph[1] ^= 1;
-          tc_fence_after();
-          if (p.want_dq2) {
+          if (G2) {
+            if (!(ok = mbar_wait(&dqempty[1], dqph[1] ^ 1, ctl))) break;
+            dqph[1] ^= 1;
+            tc_fence_after();
+            if (p.want_dq2) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma_bf16_ss(tmem_base + kColDQ2, sdesc_advance(k2m, kk * 2048),
-                           sdesc_advance(d2m, kk * 2048), idQ2, kk > 0);
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma_bf16_ss(tmem_base + kColDQ2, sdesc_advance(k2m, kk * 2048),
+                             sdesc_advance(d2m, kk * 2048), idQ2, kk > 0);
+            }
           }
           umma_commit(dqfull);
           umma_commit(&dsempty[db]);
@@ -512,14 +537,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         if (masked) {
           // first visible query (index within this half) for this key
           const int thr = p.causal ? key - off - q0 - part * QPW : -1;
-          form_ds<true>(a, b, rr, p.c1, p.c2, key_ok, thr, w1, w2);
+          form_ds<true, G1, G2>(a, b, rr, p.c1, p.c2, key_ok, thr, w1, w2);
         } else {
-          form_ds<false>(a, b, rr, p.c1, p.c2, true, 0, w1, w2);
+          form_ds<false, G1, G2>(a, b, rr, p.c1, p.c2, true, 0, w1, w2);
         }
         // the buffer is free once the contractions of the step that used it are done
         if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
         dsph[db] ^= 1;
-        store_ds(w1, w2, j, part * (QPW / 8), smem_u32(ds1_s(db)) + j * 128,
+        store_ds<G1, G2>(w1, w2, j, part * (QPW / 8), smem_u32(ds1_s(db)) + j * 128,
                  smem_u32(ds2_s(db)) + j * 128);
         fence_proxy_async_smem();
         __syncwarp();
@@ -563,8 +588,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         float* base = p.dQacc + (static_cast<size_t>(w.bh) * p.NQ + q0) * LDQ;
 #pragma unroll
         for (int tsel = 0; tsel < 2; ++tsel) {
+          if ((tsel == 0 && !G1) || (tsel == 1 && !G2)) continue;
           const bool want = tsel == 0 ? p.want_dq1 : p.want_dq2;
-          const int f = tsel == 0 ? f1 : D1 + f2;
+          const int f = tsel == 0 ? f1 : DQ2_COL + f2;
           const bool fok = (tsel == 0 ? f1 : f2) >= 0;
           const uint32_t col = tl + (tsel == 0 ? kColDQ1 : kColDQ2);
           // two halves of 32 queries; the slot is released once both are in registers
@@ -605,6 +631,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
       const bool row_ok = key < p.NK;
 #pragma unroll
       for (int tsel = 0; tsel < 2; ++tsel) {
+        if ((tsel == 0 && !G1) || (tsel == 1 && !G2)) continue;
         const bool want = tsel == 0 ? p.want_dk1 : p.want_dk2;
         if (!want) continue;
         constexpr int DMAX = D1 > D2 ? D1 : D2;
@@ -709,10 +736,10 @@ __global__ void streamkl_bwd_convert_kernel(const BwdConvertParams p) {
   }
 }
 
-template <int D1, int D2>
+template <int D1, int D2, int SEL>
 cudaError_t launch_t(const BwdParams& p, int grid, cudaStream_t stream) {
-  constexpr int smem = BwdLayout<D1, D2>::alloc;
-  auto kern = streamkl_bwd_kernel<D1, D2>;
+  constexpr int smem = BwdLayout<D1, D2, (SEL == 3) ? 2 : 1>::alloc;
+  auto kern = streamkl_bwd_kernel<D1, D2, SEL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, NTHREADS, smem, stream>>>(p);
@@ -722,18 +749,26 @@ cudaError_t launch_t(const BwdParams& p, int grid, cudaStream_t stream) {
 }  // namespace
 
 size_t bwd_smem_bytes(int d1, int d2) {
-  if (d1 == 128 && d2 == 128) return BwdLayout<128, 128>::alloc;
-  if (d1 == 128 && d2 == 64) return BwdLayout<128, 64>::alloc;
-  if (d1 == 64 && d2 == 128) return BwdLayout<64, 128>::alloc;
-  if (d1 == 64 && d2 == 64) return BwdLayout<64, 64>::alloc;
+  if (d1 == 128 && d2 == 128) return BwdLayout<128, 128, 2>::alloc;
+  if (d1 == 128 && d2 == 64) return BwdLayout<128, 64, 2>::alloc;
+  if (d1 == 64 && d2 == 128) return BwdLayout<64, 128, 2>::alloc;
+  if (d1 == 64 && d2 == 64) return BwdLayout<64, 64, 2>::alloc;
   return 0;
 }
 
-cudaError_t launch_bwd(const BwdParams& p, int d1, int d2, int grid, cudaStream_t stream) {
-  if (d1 == 128 && d2 == 128) return launch_t<128, 128>(p, grid, stream);
-  if (d1 == 128 && d2 == 64) return launch_t<128, 64>(p, grid, stream);
-  if (d1 == 64 && d2 == 128) return launch_t<64, 128>(p, grid, stream);
-  if (d1 == 64 && d2 == 64) return launch_t<64, 64>(p, grid, stream);
+template <int SEL>
+cudaError_t launch_sel(const BwdParams& p, int d1, int d2, int grid, cudaStream_t stream) {
+  if (d1 == 128 && d2 == 128) return launch_t<128, 128, SEL>(p, grid, stream);
+  if (d1 == 128 && d2 == 64) return launch_t<128, 64, SEL>(p, grid, stream);
+  if (d1 == 64 && d2 == 128) return launch_t<64, 128, SEL>(p, grid, stream);
+  if (d1 == 64 && d2 == 64) return launch_t<64, 64, SEL>(p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd(const BwdParams& p, int d1, int d2, int sel, int grid, cudaStream_t stream) {
+  if (sel == 1) return launch_sel<1>(p, d1, d2, grid, stream);
+  if (sel == 2) return launch_sel<2>(p, d1, d2, grid, stream);
+  if (sel == 3) return launch_sel<3>(p, d1, d2, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -60,7 +60,7 @@ constexpr int kRowRec = 8;
 struct BwdParams {
   CUtensorMap tmQ1, tmK1, tmQ2, tmK2;  // Q maps: 64-row boxes; K maps: 128-row boxes
   const float* rowrec;  // [BH][NQpad/64][kRowRec][64], NQpad = NQ rounded up to kBwdBQ
-  float* dQacc;         // [BH][NQ][d1 + d2] fp32, zeroed before the main kernel
+  float* dQacc;         // [BH][NQ][ld] fp32, ld = widths of the selected sides, zeroed first
   __nv_bfloat16* dK1;   // [BH][NK][d1] or null
   __nv_bfloat16* dK2;   // [BH][NK][d2] or null
   int BH, NQ, NK, NQpad, causal;
@@ -113,7 +113,9 @@ cudaError_t launch_bwd_split(const BwdSplitParams& p, BwdPass pass, int d1, int 
                              cudaStream_t stream);
 
 size_t bwd_smem_bytes(int d1, int d2);
-cudaError_t launch_bwd(const BwdParams& p, int d1, int d2, int grid, cudaStream_t stream);
+// sel: gradient sides the fused kernel forms -- 1 teacher (dQ1/dK1), 2 student
+// (dQ2/dK2), 3 both; the dQ accumulator rows hold the selected sides only.
+cudaError_t launch_bwd(const BwdParams& p, int d1, int d2, int sel, int grid, cudaStream_t stream);
 cudaError_t launch_bwd_prep(const BwdPrepParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_convert(const BwdConvertParams& p, int num_sms, cudaStream_t stream);
 

@@ -455,6 +455,10 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   const float s2 = scale_or_default(prob->s2, prob->d2);
   const bool split = resolve_bwd_algo(*prob) == STREAMKL_BWD_SPLIT;
   const bool want_dq = (dQ1 || dQ2) && !split;  // the fused path accumulates dQ in fp32
+  // Gradient sides asked for (the page's configurations): the fused kernel is
+  // specialised on them and its dQ accumulator holds only their columns.
+  const int sel = ((dQ1 || dK1) ? 1 : 0) | ((dQ2 || dK2) ? 2 : 0);
+  const int ld1 = (sel & 1) ? prob->d1 : 0, ld2 = (sel & 2) ? prob->d2 : 0;
 
   skl::BwdPrepParams pp;
   pp.L = L;
@@ -463,7 +467,7 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   pp.dL = dL;
   pp.rowrec = rowrec;
   pp.dQacc = dqacc;
-  pp.dqacc_elems = want_dq ? lay.dqacc_elems : 0;
+  pp.dqacc_elems = want_dq ? BH * static_cast<int64_t>(prob->NQ) * (ld1 + ld2) : 0;
   pp.BH = static_cast<int>(BH);
   pp.NQ = prob->NQ;
   pp.NQpad = lay.NQpad;
@@ -540,7 +544,7 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   p.wait_limit_ns = wait_limit_ns();
   const int units = skl::bwd_units(p.BH, p.NK);
   const int grid = units < dev->num_sms ? units : dev->num_sms;
-  if (skl::launch_bwd(p, prob->d1, prob->d2, grid, s) != cudaSuccess) return STREAMKL_ECUDA;
+  if (skl::launch_bwd(p, prob->d1, prob->d2, sel, grid, s) != cudaSuccess) return STREAMKL_ECUDA;
   g_launches.fetch_add(1);
 
   if (want_dq) {
@@ -549,8 +553,8 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
     cp.dQ1 = static_cast<__nv_bfloat16*>(dQ1);
     cp.dQ2 = static_cast<__nv_bfloat16*>(dQ2);
     cp.rows = BH * prob->NQ;
-    cp.d1 = prob->d1;
-    cp.d2 = prob->d2;
+    cp.d1 = ld1;  // accumulator columns: teacher side (if selected), then student side
+    cp.d2 = ld2;
     if (skl::launch_bwd_convert(cp, dev->num_sms, s) != cudaSuccess) return STREAMKL_ECUDA;
     g_launches.fetch_add(1);
   }

@@ -91,6 +91,41 @@ def test_bwd_single_output(orc):
     check_grads(gpu, oracle_heads(orc, ins, dL, False, [0]), [0], names=["dK1"])
 
 
+@pytest.mark.parametrize("need", ["1000", "0100", "0010", "0001", "1100", "0011", "1001", "0110"])
+@pytest.mark.parametrize("dims", [(128, 64), (64, 128)])
+def test_bwd_one_sided_and_partial_outputs(orc, need, dims):
+    """Every single output and both one-sided configurations, with teacher and
+    student head dimensions that differ (the one-sided kernels keep a dQ
+    accumulator of one side's width), ragged non-causal tiles."""
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(1, 2, 136, 200, dims[0], dims[1], False)
+    ins = make_inputs(w)
+    dL = torch.randn((w.B, w.H, w.NQ), generator=torch.Generator().manual_seed(15))
+    nd = tuple(c == "1" for c in need)
+    gpu = run_bwd(cuda_inputs(ins), dL.cuda(), False, need=nd)
+    assert [g is None for g in gpu] == [not x for x in nd]
+    names = [n for n, x in zip(("dQ1", "dK1", "dQ2", "dK2"), nd) if x]
+    check_grads(gpu, oracle_heads(orc, ins, dL, False, [0, 1]), [0, 1], names=names)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_one_sided_dk_matches_full_kernel_bitwise(bwd_algo, causal):
+    """dK is accumulated in TMEM in a fixed order, and a one-sided kernel forms
+    its dS with the same arithmetic as the two-sided one, so its dK is the
+    same to the bit (dQ goes through fp32 atomics and is not compared)."""
+    if bwd_algo != "fused":
+        pytest.skip("the specialised kernels are the fused path")
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(1, 2, 192, 320, 128, 128, causal)
+    dev = cuda_inputs(make_inputs(w))
+    dL = torch.randn((1, 2, w.NQ), device="cuda")
+    full = run_bwd(dev, dL, causal)
+    teacher = run_bwd(dev, dL, causal, need=(False, True, False, False))
+    student = run_bwd(dev, dL, causal, need=(False, False, False, True))
+    assert np.array_equal(teacher[1], full[1])
+    assert np.array_equal(student[3], full[3])
+
+
 def test_bwd_explicit_scales(orc):
     from attention_kl_distillation_b200.inputs import make_inputs
     w = workload(1, 1, 128, 192, 128, 128, True)
