@@ -17,6 +17,7 @@ constexpr int kFwdBK = 128;
 
 struct FwdParams {
   CUtensorMap tmK1, tmK2;  // 3-D maps over [BH][NK][d], 128-row boxes, 128B swizzle
+  CUtensorMap tmQ1, tmQ2;  // transposed kernel only: [BH][NQ][d], boxes of one query group
   const __nv_bfloat16* Q1;  // [BH][NQ][d1], read row by row into TMEM
   const __nv_bfloat16* Q2;  // [BH][NQ][d2]
   float* L;
@@ -49,6 +50,17 @@ size_t fwd_smem_bytes(int d1, int d2);
 
 // Launch the forward kernel; returns the launch error.
 cudaError_t launch_fwd(const FwdParams& p, int d1, int d2, int grid, cudaStream_t stream);
+
+// Transposed forward for few query rows (keys on the UMMA M axis): problems
+// with NQ <= kFwdTMaxNQ use it; the rows form query groups of fwd_t_rows(NQ)
+// (the UMMA N), and a work unit is (bh, group, key split).
+constexpr int kFwdTMaxNQ = 32;
+__host__ __device__ inline int fwd_t_rows(int NQ) { return NQ <= 16 ? 16 : 32; }
+__host__ __device__ inline int fwd_t_units(int BH, int NQ, int nsplit = 1) {
+  const int nqt = fwd_t_rows(NQ);
+  return BH * ((NQ + nqt - 1) / nqt) * (nsplit > 1 ? nsplit : 1);
+}
+cudaError_t launch_fwd_t(const FwdParams& p, int d1, int d2, int nqt, int grid, cudaStream_t stream);
 
 // Keys per backward work unit (UMMA M of S^T and dK) and queries per step.
 constexpr int kBwdBK = 128;

@@ -264,13 +264,30 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
 }
 
 // 32 lanes x N consecutive 32-bit columns, N = 16 or 32.
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+
 template <int N>
 __device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, uint32_t (&r)[N]) {
-  static_assert(N == 16 || N == 32, "16 or 32 columns");
+  static_assert(N == 4 || N == 8 || N == 16 || N == 32, "4, 8, 16 or 32 columns");
   if constexpr (N == 32) {
     tmem_ld_32x32b_x32(taddr, r);
-  } else {
+  } else if constexpr (N == 16) {
     tmem_ld_32x32b_x16(taddr, r);
+  } else if constexpr (N == 8) {
+    tmem_ld_32x32b_x8(taddr, r);
+  } else {
+    tmem_ld_32x32b_x4(taddr, r);
   }
 }
 

@@ -297,6 +297,11 @@ streamkl_status prepare_fwd(const streamkl_problem* prob, const void* Q1, const 
   const int64_t BH = static_cast<int64_t>(prob->B) * prob->H;
   if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kFwdBK, &p->tmK1)) != STREAMKL_OK) return st;
   if ((st = tensor_map(K2, BH, prob->NK, prob->d2, skl::kFwdBK, &p->tmK2)) != STREAMKL_OK) return st;
+  if (prob->NQ <= skl::kFwdTMaxNQ) {  // transposed kernel: Q groups are TMA boxes
+    const int nqt = skl::fwd_t_rows(prob->NQ);
+    if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, nqt, &p->tmQ1)) != STREAMKL_OK) return st;
+    if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, nqt, &p->tmQ2)) != STREAMKL_OK) return st;
+  }
   p->Q1 = static_cast<const __nv_bfloat16*>(Q1);
   p->Q2 = static_cast<const __nv_bfloat16*>(Q2);
   p->L = L;
@@ -320,6 +325,21 @@ streamkl_status prepare_fwd(const streamkl_problem* prob, const void* Q1, const 
 
 int fwd_key_tiles(const streamkl_problem& pr) { return (pr.NK + skl::kFwdBK - 1) / skl::kFwdBK; }
 
+// The forward kernel for a problem: few query rows go to the transposed
+// kernel (keys on the UMMA M axis), the rest to the 128-row tile kernel.
+bool fwd_transposed(const streamkl_problem& pr) { return pr.NQ <= skl::kFwdTMaxNQ; }
+
+int fwd_unit_count(const streamkl_problem& pr, int nsplit) {
+  const int BH = pr.B * pr.H;
+  return fwd_transposed(pr) ? skl::fwd_t_units(BH, pr.NQ, nsplit) : skl::fwd_units(BH, pr.NQ, nsplit);
+}
+
+cudaError_t launch_fwd_any(const streamkl_problem& pr, const skl::FwdParams& p, int grid,
+                           cudaStream_t s) {
+  if (fwd_transposed(pr)) return skl::launch_fwd_t(p, pr.d1, pr.d2, skl::fwd_t_rows(pr.NQ), grid, s);
+  return skl::launch_fwd(p, pr.d1, pr.d2, grid, s);
+}
+
 // Key tiles per chunk and the effective chunk count for a requested split.
 void split_shape(const streamkl_problem& pr, int nsplit, int* kt_chunk, int* nsp) {
   const int nkt = fwd_key_tiles(pr);
@@ -341,10 +361,9 @@ streamkl_status streamkl_fwd(const streamkl_problem* prob, const void* Q1, const
   DeviceInfo* dev = nullptr;
   streamkl_status st = prepare_fwd(prob, Q1, K1, Q2, K2, L, LSE1, LSE2, &p, &dev);
   if (st != STREAMKL_OK) return st;
-  const int units = skl::fwd_units(p.BH, p.NQ);
+  const int units = fwd_unit_count(*prob, 1);
   const int grid = units < dev->num_sms ? units : dev->num_sms;
-  if (skl::launch_fwd(p, prob->d1, prob->d2, grid, reinterpret_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  if (launch_fwd_any(*prob, p, grid, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STREAMKL_ECUDA;
   g_launches.fetch_add(1);
   return STREAMKL_OK;
@@ -362,13 +381,18 @@ int streamkl_fwd_splitk_suggest(const streamkl_problem* prob) {
   if (check_problem(prob) != STREAMKL_OK) return 0;
   DeviceInfo* dev = nullptr;
   if (current_device(&dev) != STREAMKL_OK) return 0;
-  const int units = skl::fwd_units(prob->B * prob->H, prob->NQ);
-  const int want = 2 * dev->num_sms;
-  if (units >= dev->num_sms) return 1;
-  int n = (want + units - 1) / units;
+  const int units = fwd_unit_count(*prob, 1);
+  const int sms = dev->num_sms;
+  if (units >= sms) return 1;
+  // About four units per SM: measured on B200 for B1 H32 NK=32768 (32 and 64
+  // unsplit units), fewer splits leave HBM idle in the last waves and more add
+  // per-unit work (Q load, lane merge) and merge traffic.
+  int n = (4 * sms) / units;
   const int nkt = fwd_key_tiles(*prob);
   if (n > nkt) n = nkt;
-  return n < 1 ? 1 : n;
+  int chunk, best;
+  split_shape(*prob, n < 1 ? 1 : n, &chunk, &best);
+  return best < 1 ? 1 : best;
 }
 
 streamkl_status streamkl_fwd_splitk(const streamkl_problem* prob, const void* Q1, const void* K1,
@@ -392,9 +416,9 @@ streamkl_status streamkl_fwd_splitk(const streamkl_problem* prob, const void* Q1
     p.nsplit = nsp;
     p.part = static_cast<float*>(workspace);
   }
-  const int units = skl::fwd_units(p.BH, p.NQ, p.nsplit);
+  const int units = fwd_unit_count(*prob, p.nsplit);
   const int grid = units < dev->num_sms ? units : dev->num_sms;
-  if (skl::launch_fwd(p, prob->d1, prob->d2, grid, s) != cudaSuccess) return STREAMKL_ECUDA;
+  if (launch_fwd_any(*prob, p, grid, s) != cudaSuccess) return STREAMKL_ECUDA;
   g_launches.fetch_add(1);
   if (nsp > 1) {
     skl::FwdMergeParams mp;

@@ -70,7 +70,10 @@ typedef struct {
  * Section 1 of the page: the five running scalars m1, m2, l1, l2 and acc per
  * row, finished as L = acc/l1 + LSE2 - LSE1 with LSE_t = m_t + log l_t; key
  * tiles past the causal frontier are skipped.  L, LSE1 and LSE2 are also
- * the saved state of section 2 that streamkl_bwd consumes.
+ * the saved state of section 2 that streamkl_bwd consumes.  Problems with
+ * NQ <= 32 run a transposed kernel (keys on the MMA's long axis, as in the
+ * ETAP page's S^T = K Q^T); the results agree with the row-tile kernel to
+ * fp32 rounding.
  * Errors: EINVAL (null or unaligned pointer, sizes out of range, causal with
  * NQ > NK), EUNSUPPORTED (d not in {64,128}, device is not sm_100), ECUDA.
  */
@@ -100,9 +103,9 @@ streamkl_status streamkl_fwd_splitk(const streamkl_problem *prob, const void *Q1
 size_t streamkl_fwd_splitk_workspace_size(const streamkl_problem *prob, int nsplit);
 
 /*
- * A split count for the current device: enough key chunks that the forward's
- * work units fill every SM about twice; 1 when the problem already does.
- * 0 on a bad problem or if the device cannot be queried.
+ * A split count for the current device: about four of the forward's work
+ * units per SM (at most one key tile per chunk); 1 when the problem already
+ * has a unit per SM.  0 on a bad problem or if the device cannot be queried.
  */
 int streamkl_fwd_splitk_suggest(const streamkl_problem *prob);
 

@@ -13,7 +13,8 @@ def test_inject_argument_validation():
 
 
 @pytest.mark.gpu
-def test_stalled_producer_times_out_and_context_survives():
+@pytest.mark.parametrize("nq", [300, 20], ids=["row_tiles", "transposed"])
+def test_stalled_producer_times_out_and_context_survives(nq):
     import numpy as np
     import torch
 
@@ -21,7 +22,7 @@ def test_stalled_producer_times_out_and_context_survives():
     from attention_kl_distillation_b200.inputs import make_inputs
     from gpu_common import cuda_inputs, workload
 
-    w = workload(1, 2, 300, 300, 128, 128, True)
+    w = workload(1, 2, nq, 300, 128, 128, True)
     dev = cuda_inputs(make_inputs(w))
     torch.cuda.synchronize()
     assert query_device_status() == B.OK
