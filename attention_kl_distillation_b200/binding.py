@@ -200,6 +200,15 @@ def fwd_splitk(Q1, K1, Q2, K2, causal=False, s1=None, s2=None, nsplit=None, work
     return L, A, Bv
 
 
+def splitk_suggest(B, H, NQ, NK, d1, d2, causal=False) -> int:
+    """streamkl_fwd_splitk_suggest for the current device."""
+    prob = problem(B, H, NQ, NK, d1, d2, causal)
+    n = int(_lib.streamkl_fwd_splitk_suggest(ctypes.byref(prob)))
+    if n < 1:
+        raise StreamKLError(EINVAL, "streamkl_fwd_splitk_suggest")
+    return n
+
+
 def workspace_size(B, H, NQ, NK, d1, d2, causal=False) -> int:
     prob = problem(B, H, NQ, NK, d1, d2, causal)
     return int(_lib.streamkl_bwd_workspace_size(ctypes.byref(prob)))

@@ -56,6 +56,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (smaller cases for profiling; not a bench line)")
+    ap.add_argument("--nq", type=int, default=None,
+                    help="override NQ (small-NQ forward cases; not a bench line)")
+    ap.add_argument("--splitk", action="store_true",
+                    help="run the forward through streamkl_fwd_splitk with the suggested split")
     ap.add_argument("--need", default="1111",
                     help="which of dQ1 dK1 dQ2 dK2 the backward returns (e.g. 0101 = dK only)")
     return ap.parse_args(argv)
@@ -250,6 +254,8 @@ def main(argv=None):
     w = WORKLOADS[args.workload]
     if args.heads:
         w = w.with_(H=args.heads)
+    if args.nq:
+        w = w.with_(NQ=args.nq)
     phase = args.phase if args.phase != "auto" else ("fwdbwd" if w.backward else "fwd")
     if args.impl == "reference":
         return run_reference(args, w, phase)
@@ -280,9 +286,20 @@ def main(argv=None):
     grads = tuple(torch.empty_like(t) if n else None for t, n in zip((Q1, K1, Q2, K2), need))
     ws = torch.empty(binding.workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal),
                      dtype=torch.uint8, device=dev)
+    nsplit = None
+    if args.splitk:
+        nsplit = binding.splitk_suggest(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal)
+        fws = torch.empty(max(256, binding.splitk_workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, nsplit)),
+                          dtype=torch.uint8, device=dev)
+
+    def fwd_call():
+        if nsplit is None:
+            skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B))
+        else:
+            skl.fwd_splitk(Q1, K1, Q2, K2, causal=w.causal, nsplit=nsplit, workspace=fws, out=(L, A, B))
 
     def step():
-        skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B))
+        fwd_call()
         if phase == "fwdbwd":
             skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal, workspace=ws, out=grads)
 
@@ -309,7 +326,7 @@ def main(argv=None):
     t_start.record(stream)
     for k in range(args.steps):
         ev[k][0].record(stream)
-        skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B))
+        fwd_call()
         ev[k][1].record(stream)
         if phase == "fwdbwd":
             skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal, workspace=ws, out=grads)
@@ -345,6 +362,15 @@ def main(argv=None):
                 "frac": dom["achieved"] / peak, "traffic": dom["traffic"], "kernel": dom["kernel"],
                 "flops_per_launch": dom["flops_per_launch"], "ms_per_launch": dom["ms"],
                 "peak_source": f"{src} dense bf16 (burst)"}
+    if phase == "fwd" and w.NQ <= 32:
+        # few query rows: the transposed kernel streams K1 and K2 once per head; the
+        # algorithmic bytes are the inputs read once plus the three fp32 row vectors
+        alg = w.input_bytes() + 3 * w.BH * w.NQ * 4
+        gbs = alg / (fwd_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                    "traffic": None,
+                    "kernel": "streamkl_fwd_t_kernel" + (" + streamkl_fwd_merge_kernel" if nsplit else ""),
+                    "bytes_per_launch": alg, "ms_per_launch": fwd_ms, "peak_source": f"{src} HBM copy"}
 
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -399,6 +425,7 @@ def main(argv=None):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) teacher, student = teacher + noise; bf16)",
         "config": {**workload_desc(w, phase), **({"need": args.need} if args.need != "1111" else {}),
+                   **({"splitk": nsplit} if nsplit else {}),
                    "parallelism": f"dp{world} (independent replicas, no collective)"},
         "pct_of_peak": value / world / peak,
         "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac_of_peak": fwd_tf / peak,
