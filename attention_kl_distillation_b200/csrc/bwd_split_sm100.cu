@@ -14,7 +14,9 @@
 // Both have the same shape, OUT += dS . C with dS = f(R C^T): S (M=128, N=64)
 // comes from a UMMA with both operands in shared memory, dS is written in bf16
 // to TMEM by the compute warps and the product is a UMMA whose A operand is
-// that TMEM tile.  Each pass regenerates P1, P2 from the saved LSEs and keeps
+// that TMEM tile.  S of successive steps alternates between two TMEM slots and
+// dS is written into the slot it came from, so S of step t+1 is computed while
+// dS of step t is formed and contracted.  Each pass regenerates P1, P2 from the saved LSEs and keeps
 // its gradient in TMEM for the whole unit, so no accumulator in global memory
 // and no atomics are needed; the price is recomputing S and the exponentials
 // once more than the fused kernel does.
@@ -23,8 +25,12 @@
 // dK pass the per-query records of each step) and unit dispenser; warp 1 TMEM
 // owner and UMMA issuer; warps 2..17 four compute warpgroups, each owning 16 of
 // the 64 streamed rows of a step (thread = resident row = TMEM lane).
-// TMEM: S1 [0,64) S2 [64,128) dS (bf16, two buffers of 32+32) [128,256)
-//       OUT1 [256, 256+d1) OUT2 [256+d1, 256+d1+d2).
+// TMEM: two slots of 128 columns at 0 and 128, each S1 [0,64) S2 [64,128) of
+//       one step; OUT1 [256, 256+d1) OUT2 [256+d1, 256+d1+d2).  A compute
+//       warpgroup that owns streamed rows [16p, 16p+16) reads S1 columns
+//       [16p, 16p+16) of the slot and writes its bf16 dS1 and dS2 over them
+//       ([16p, 16p+8) and [16p+8, 16p+16)): columns only it has read, and the
+//       eight columns one K16 step of the product reads as its A operand.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -39,7 +45,7 @@ constexpr int NDS = 4;                      // compute warpgroups
 constexpr int CPW = CB / NDS;               // streamed rows per compute warpgroup
 constexpr int NTHREADS = (2 + 4 * NDS) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr uint32_t kColS1 = 0, kColS2 = 64, kColDS = 128, kColOut = 256;
+constexpr uint32_t kSlotCols = 128, kColS2 = 64, kColOut = 256;
 constexpr int kNegInf = -(1 << 30), kPosInf = (1 << 30);
 
 template <BwdPass PASS, int D1, int D2>
@@ -55,9 +61,8 @@ struct SplitLayout {
   static constexpr int nst_fit = (232448 - 1024 - 512 - c_off) / stage_bytes;
   static constexpr int NST = nst_fit > 6 ? 6 : nst_fit;
   static constexpr int bar_off = c_off + NST * stage_bytes;
-  // rfull rempty cfull[NST] cempty[NST] sfull sempty dsfull[2] dsempty[2] ofull oempty
-  // ufull[2] uempty[2] drain
-  static constexpr int nbar = 2 + 2 * NST + 2 + 4 + 2 + 4 + 1;
+  // rfull rempty cfull[NST] cempty[NST] sfull[2] dsfull[2] ofull oempty ufull[2] uempty[2] drain
+  static constexpr int nbar = 2 + 2 * NST + 4 + 2 + 4 + 1;
   static constexpr int misc_off = bar_off + nbar * 8;
   static constexpr int alloc = misc_off + 32 + 1024;
   static_assert(NST >= 3, "streamed ring too shallow");
@@ -192,11 +197,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* rempty = bars + 1;
   uint64_t* cfull = bars + 2;
   uint64_t* cempty = cfull + NST;
-  uint64_t* sfull = cempty + NST;
-  uint64_t* sempty = sfull + 1;
-  uint64_t* dsfull = sempty + 1;  // [2]
-  uint64_t* dsempty = dsfull + 2;  // [2]
-  uint64_t* ofull = dsempty + 2;
+  uint64_t* sfull = cempty + NST;  // [2]: S of a step is in the slot
+  uint64_t* dsfull = sfull + 2;    // [2]: dS of a step has replaced it
+  uint64_t* ofull = dsfull + 2;
   uint64_t* oempty = ofull + 1;
   uint64_t* ufull = oempty + 1;  // [2]
   uint64_t* uempty = ufull + 2;  // [2]
@@ -217,11 +220,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&cfull[s], 1);
       mbar_init(&cempty[s], 1);
     }
-    mbar_init(sfull, 1);
-    mbar_init(sempty, 4 * NDS);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&sfull[s], 1);
       mbar_init(&dsfull[s], 4 * NDS);
-      mbar_init(&dsempty[s], 1);
       mbar_init(&ufull[s], 1);
       mbar_init(&uempty[s], 1 + 4 * NDS);  // MMA thread + compute warps
     }
@@ -322,9 +323,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr uint32_t idO2 = idesc_bf16(RB, D2, 0, 1);
       const uint64_t r1d = sdesc_sw128(smem_u32(r1_s), 16, 1024);
       const uint64_t r2d = sdesc_sw128(smem_u32(r2_s), 16, 1024);
-      int us = 0, cs_s = 0, cs_r = 0, db = 0;
-      uint32_t uph = 0, rph = 0, cph_s = 0, sph = 0, oph = 0;
-      uint32_t dsph[2] = {0, 0};
+      // slot_s: the slot the next S goes to; slot_r: the slot of the step whose
+      // product is next.  A slot's S is issued only after the product that read
+      // its previous dS (UMMAs of this thread execute in issue order).
+      int us = 0, cs_s = 0, cs_r = 0, slot_s = 0, slot_r = 0;
+      uint32_t uph = 0, rph = 0, cph_s = 0, oph = 0;
+      uint32_t dsph = 0;  // bit s: parity of slot s's dsfull
       bool ok = true;
       for (;;) {
         if (!(ok = mbar_wait(&ufull[us], uph, ctl))) break;
@@ -340,24 +344,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         rph ^= 1;
         auto issue_s = [&]() -> bool {
           if (!mbar_wait(&cfull[cs_s], cph_s, ctl)) return false;
-          if (!mbar_wait(sempty, sph ^ 1, ctl)) return false;
           tc_fence_after();
+          const uint32_t sd = tmem_base + slot_s * kSlotCols;
           const uint64_t c1d = sdesc_sw128(smem_u32(c1_s(cs_s)), 16, 1024);
           const uint64_t c2d = sdesc_sw128(smem_u32(c2_s(cs_s)), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D1 / 16; ++kk) {
             const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(tmem_base + kColS1, sdesc_advance(r1d, (kk >> 2) * (RB * 128) + o),
+            umma_bf16_ss(sd, sdesc_advance(r1d, (kk >> 2) * (RB * 128) + o),
                          sdesc_advance(c1d, (kk >> 2) * (CB * 128) + o), idS, kk > 0);
           }
 #pragma unroll
           for (int kk = 0; kk < D2 / 16; ++kk) {
             const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(tmem_base + kColS2, sdesc_advance(r2d, (kk >> 2) * (RB * 128) + o),
+            umma_bf16_ss(sd + kColS2, sdesc_advance(r2d, (kk >> 2) * (RB * 128) + o),
                          sdesc_advance(c2d, (kk >> 2) * (CB * 128) + o), idS, kk > 0);
           }
-          umma_commit(sfull);
-          sph ^= 1;
+          umma_commit(&sfull[slot_s]);
+          slot_s ^= 1;
           if (++cs_s == NST) {
             cs_s = 0;
             cph_s ^= 1;
@@ -367,8 +371,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!(ok = issue_s())) break;
         for (int t = 0; t < w.nsteps && ok; ++t) {
           if (t + 1 < w.nsteps && !(ok = issue_s())) break;
-          if (!(ok = mbar_wait(&dsfull[db], dsph[db], ctl))) break;
-          dsph[db] ^= 1;
+          if (!(ok = mbar_wait(&dsfull[slot_r], (dsph >> slot_r) & 1u, ctl))) break;
+          dsph ^= 1u << slot_r;
           if (t == 0) {
             if (!(ok = mbar_wait(oempty, oph ^ 1, ctl))) break;
             oph ^= 1;
@@ -377,21 +381,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // C tiles read MN-major: features contiguous, 64-feature chunks 8 KB apart
           const uint64_t c1m = sdesc_sw128(smem_u32(c1_s(cs_r)), CB * 128, 1024);
           const uint64_t c2m = sdesc_sw128(smem_u32(c2_s(cs_r)), CB * 128, 1024);
-          const uint32_t dsa = tmem_base + kColDS + db * 64;
-          // OUT_t += dS_t (TMEM, 64 streamed rows along K, 8 columns per 16) . C_t
-          // (read MN-major: features contiguous, 64-feature chunks 8 KB apart).
+          const uint32_t dsa = tmem_base + slot_r * kSlotCols;
+          // OUT_t += dS_t (TMEM; K16 step kk: dS1 in columns [16kk, 16kk+8), dS2 in
+          // [16kk+8, 16kk+16) of the slot) . C_t (read MN-major: features
+          // contiguous, 64-feature chunks 8 KB apart).
 #pragma unroll
           for (int kk = 0; kk < CB / 16; ++kk) {
             if (p.out1)
-              umma_bf16_ts(tmem_base + kColOut, dsa + kk * 8, sdesc_advance(c1m, kk * 2048), idO1,
+              umma_bf16_ts(tmem_base + kColOut, dsa + kk * 16, sdesc_advance(c1m, kk * 2048), idO1,
                            (t > 0 || kk > 0));
             if (p.out2)
-              umma_bf16_ts(tmem_base + kColOut + D1, dsa + 32 + kk * 8, sdesc_advance(c2m, kk * 2048),
+              umma_bf16_ts(tmem_base + kColOut + D1, dsa + kk * 16 + 8, sdesc_advance(c2m, kk * 2048),
                            idO2, (t > 0 || kk > 0));
           }
-          umma_commit(&dsempty[db]);
           umma_commit(&cempty[cs_r]);
-          db ^= 1;
+          slot_r ^= 1;
           if (++cs_r == NST) cs_r = 0;
         }
         if (!ok) break;
@@ -409,9 +413,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int quarter = warp & 3;
     const int j = quarter * 32 + lane;  // resident row within the tile (TMEM lane)
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    int us = 0, cs = 0, db = 0;
-    uint32_t uph = 0, cph = 0, sph = 0, oph = 0;
-    uint32_t dsph[2] = {0, 0};
+    int us = 0, cs = 0, slot = 0;
+    uint32_t uph = 0, cph = 0, oph = 0;
+    uint32_t sph = 0;  // bit s: parity of slot s's sfull
     bool ok = true;
     for (;;) {
       if (!(ok = mbar_wait(&ufull[us], uph, ctl))) break;
@@ -437,18 +441,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (DK) {
           if (!(ok = mbar_wait(&cfull[cs], cph, ctl))) break;  // per-query records of the step
         }
-        if (!(ok = mbar_wait(sfull, sph, ctl))) break;
-        sph ^= 1;
+        if (!(ok = mbar_wait(&sfull[slot], (sph >> slot) & 1u, ctl))) break;
+        sph ^= 1u << slot;
         tc_fence_after();
+        const uint32_t scol = tl + slot * kSlotCols + part * CPW;
         uint32_t a[CPW], b[CPW];
-        tmem_ld_32x32b_x16(tl + kColS1 + part * CPW, a);
-        tmem_ld_32x32b_x16(tl + kColS2 + part * CPW, b);
+        tmem_ld_32x32b_x16(scol, a);
+        tmem_ld_32x32b_x16(scol + kColS2, b);
         tmem_ld_wait();
         reg_fence(a);
         reg_fence(b);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sempty);
         const int c0 = w.c0(t);
         bool masked;
         int lo = kNegInf, hi = kPosInf;
@@ -467,16 +469,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           form_ds<true, DK>(a, b, rr, rec, p.c1, p.c2, lo, hi, w1, w2);
         else
           form_ds<false, DK>(a, b, rr, rec, p.c1, p.c2, lo, hi, w1, w2);
-        if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
-        dsph[db] ^= 1;
-        const uint32_t dsa = tl + kColDS + db * 64 + part * (CPW / 2);
-        tmem_st_32x32b_x8(dsa, w1);
-        tmem_st_32x32b_x8(dsa + 32, w2);
+        // dS over this warpgroup's own S1 columns of the slot
+        tmem_st_32x32b_x8(scol, w1);
+        tmem_st_32x32b_x8(scol + CPW / 2, w2);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dsfull[db]);
-        db ^= 1;
+        if (lane == 0) mbar_arrive(&dsfull[slot]);
+        slot ^= 1;
         if (++cs == NST) {
           cs = 0;
           cph ^= 1;

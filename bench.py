@@ -372,44 +372,66 @@ def main(argv=None):
                     "kernel": "streamkl_fwd_t_kernel" + (" + streamkl_fwd_merge_kernel" if nsplit else ""),
                     "bytes_per_launch": alg, "ms_per_launch": fwd_ms, "peak_source": f"{src} HBM copy"}
 
-    # end to end through the public API: pinned host inputs in, result out, every step
+    # End to end through the public API: every step copies its inputs from pinned
+    # host memory and reads its result (the per-row KL) back to the host.  The copy
+    # of step k+1's inputs runs on a side stream into the other of two device
+    # buffers while step k computes (the loader prefetch a training loop has); the
+    # gradients stay on the device, where an optimizer would consume them.
     e2e = None
     if not args.no_e2e:
         h_in = [t.pin_memory() for t in cpu_ins]
         h_dL = dL.cpu().pin_memory()
         h_L = torch.empty((w.B, w.H, w.NQ), dtype=torch.float32).pin_memory()
-        h_g = [torch.empty(t.shape, dtype=torch.bfloat16).pin_memory() for t in cpu_ins]
         h2d = sum(t.numel() * t.element_size() for t in h_in) + h_dL.numel() * 4
-        d2h = h_L.numel() * 4 + (sum(t.numel() * 2 for t in h_g) if phase == "fwdbwd" else 0)
+        d2h = h_L.numel() * 4
+        bufs = [[torch.empty_like(t, device=dev) for t in cpu_ins] + [torch.empty_like(dL)]
+                for _ in range(2)]
+        copy_stream = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        used = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            d_in = [t.to(dev, non_blocking=True) for t in h_in]
-            d_dL = h_dL.to(dev, non_blocking=True)
-            if phase == "fwdbwd":
-                Lx = skl.streamkl(*[t.requires_grad_(True) for t in d_in], causal=w.causal)
-                Lx.backward(d_dL)
-                for hg, t in zip(h_g, d_in):
-                    hg.copy_(t.grad, non_blocking=True)
-            else:
-                Lx, _, _ = skl.fwd(*d_in, causal=w.causal)
-            h_L.copy_(Lx.detach(), non_blocking=True)
+        def e2e_run(n, start=None):
+            """n steps; returns nothing.  Copies for step k go to buffer k % 2."""
+            def issue_copy(k):
+                b = k % 2
+                with torch.cuda.stream(copy_stream):
+                    if k >= 2:
+                        copy_stream.wait_event(used[b])  # step k-2 is done with the buffer
+                    for dst, src in zip(bufs[b], h_in + [h_dL]):
+                        dst.copy_(src, non_blocking=True)
+                    copied[b].record(copy_stream)
+            if start is not None:
+                copy_stream.wait_event(start)
+            issue_copy(0)
+            for k in range(n):
+                if k + 1 < n:
+                    issue_copy(k + 1)
+                b = k % 2
+                stream.wait_event(copied[b])
+                d_in = [t.detach().requires_grad_(phase == "fwdbwd") for t in bufs[b][:4]]
+                if phase == "fwdbwd":
+                    Lx = skl.streamkl(*d_in, causal=w.causal)
+                    Lx.backward(bufs[b][4])
+                else:
+                    Lx, _, _ = skl.fwd(*d_in, causal=w.causal)
+                h_L.copy_(Lx.detach(), non_blocking=True)
+                used[b].record(stream)
 
-        for _ in range(2):
-            e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize()
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         ke = max(3, min(args.steps, 10))
         e0.record(stream)
-        for _ in range(ke):
-            e2e_step()
+        e2e_run(ke, start=e0)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
         e2e = {"value": world * fl_step * ke / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_ms / ke, "api": "attention_kl_distillation_b200.streamkl"}
+               "ms_per_step": e2e_ms / ke, "api": "attention_kl_distillation_b200.streamkl",
+               "pipeline": "inputs of step k+1 copied on a side stream during step k; result L read back every step"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
