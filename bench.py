@@ -96,28 +96,41 @@ def workload_desc(w: Workload, phase: str) -> dict:
     }
 
 
-def kernel_sources_sha1() -> str:
+# The sources a profiled kernel is built from: its own file and the two shared headers.
+PROFILED_SOURCES = {
+    "fwd_kernel": "fwd_sm100.cu",
+    "fwd_t_kernel": "fwd_t_sm100.cu",
+    "bwd_fused_kernel": "bwd_sm100.cu",
+    "bwd_split_kernel": "bwd_split_sm100.cu",
+}
+
+
+def kernel_sources_sha1(kernel_file: str) -> str:
     import hashlib
     h = hashlib.sha1()
     csrc = ROOT / "attention_kl_distillation_b200" / "csrc"
-    for f in sorted(csrc.iterdir()):
-        if f.suffix in (".cu", ".cuh", ".h"):
-            h.update(f.name.encode())
-            h.update(f.read_bytes())
+    for name in (kernel_file, "kernels.h", "sm100.cuh"):
+        f = csrc / name
+        h.update(f.name.encode())
+        h.update(f.read_bytes())
     return h.hexdigest()
 
 
 def profiled_traffic(profile: str):
-    """DRAM bytes per full launch recorded in profiles/<profile>, or None when the kernel
-    sources changed since that ncu capture."""
+    """DRAM bytes per full launch recorded in profiles/<profile>, or None when the
+    kernel's sources changed since that ncu capture."""
     import re
     f = ROOT / "profiles" / profile
     if not f.exists():
         return None
+    kernel = next((k for k in sorted(PROFILED_SOURCES, key=len, reverse=True)
+                   if profile.startswith(k + "_")), None)
+    if kernel is None:
+        return None
     text = f.read_text()
     m1 = re.search(r"source-sha1: ([0-9a-f]{40})", text)
     m2 = re.search(r"dram-bytes-per-full-launch: (\d+)", text)
-    if not (m1 and m2) or m1.group(1) != kernel_sources_sha1():
+    if not (m1 and m2) or m1.group(1) != kernel_sources_sha1(PROFILED_SOURCES[kernel]):
         return None
     return int(m2.group(1))
 
@@ -367,8 +380,9 @@ def main(argv=None):
         # algorithmic bytes are the inputs read once plus the three fp32 row vectors
         alg = w.input_bytes() + 3 * w.BH * w.NQ * 4
         gbs = alg / (fwd_ms * 1e-3) / 1e9
+        captured = args.workload == "long64k" and w.NQ == 1 and nsplit is not None and not args.heads
         roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                    "traffic": None,
+                    "traffic": profiled_traffic("fwd_t_kernel_long64k_nq1.md") if captured else None,
                     "kernel": "streamkl_fwd_t_kernel" + (" + streamkl_fwd_merge_kernel" if nsplit else ""),
                     "bytes_per_launch": alg, "ms_per_launch": fwd_ms, "peak_source": f"{src} HBM copy"}
 
