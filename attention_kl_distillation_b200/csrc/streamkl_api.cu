@@ -329,9 +329,16 @@ int fwd_key_tiles(const streamkl_problem& pr) { return (pr.NK + skl::kFwdBK - 1)
 // kernel (keys on the UMMA M axis), the rest to the 128-row tile kernel.
 bool fwd_transposed(const streamkl_problem& pr) { return pr.NQ <= skl::kFwdTMaxNQ; }
 
+// Forward work units, in 64 bits: the kernels count units in int, so a launch
+// whose count does not fit is refused (EINVAL) before it is made.
+int64_t fwd_unit_count64(const streamkl_problem& pr, int nsplit) {
+  const int64_t BH = static_cast<int64_t>(pr.B) * pr.H;
+  const int rows = fwd_transposed(pr) ? skl::fwd_t_rows(pr.NQ) : skl::kFwdBQ;
+  return BH * ((pr.NQ + rows - 1) / rows) * (nsplit > 1 ? nsplit : 1);
+}
+
 int fwd_unit_count(const streamkl_problem& pr, int nsplit) {
-  const int BH = pr.B * pr.H;
-  return fwd_transposed(pr) ? skl::fwd_t_units(BH, pr.NQ, nsplit) : skl::fwd_units(BH, pr.NQ, nsplit);
+  return static_cast<int>(fwd_unit_count64(pr, nsplit));
 }
 
 cudaError_t launch_fwd_any(const streamkl_problem& pr, const skl::FwdParams& p, int grid,
@@ -361,6 +368,7 @@ streamkl_status streamkl_fwd(const streamkl_problem* prob, const void* Q1, const
   DeviceInfo* dev = nullptr;
   streamkl_status st = prepare_fwd(prob, Q1, K1, Q2, K2, L, LSE1, LSE2, &p, &dev);
   if (st != STREAMKL_OK) return st;
+  if (fwd_unit_count64(*prob, 1) > INT32_MAX) return STREAMKL_EINVAL;
   const int units = fwd_unit_count(*prob, 1);
   const int grid = units < dev->num_sms ? units : dev->num_sms;
   if (launch_fwd_any(*prob, p, grid, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -410,6 +418,7 @@ streamkl_status streamkl_fwd_splitk(const streamkl_problem* prob, const void* Q1
   if (st != STREAMKL_OK) return st;
   int chunk, nsp;
   split_shape(*prob, nsplit, &chunk, &nsp);
+  if (fwd_unit_count64(*prob, nsp) > INT32_MAX) return STREAMKL_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (nsp > 1) {
     p.kt_chunk = chunk;

@@ -86,3 +86,19 @@ def test_transposed_splitk(orc, shape, nsplit):
     gpu = tuple(t.reshape(w.BH, -1).cpu().numpy().astype(np.float64) for t in (L, A, B))
     rows = all_rows(w.BH, w.NQ)
     check_fwd(gpu, orc.fwd_rows(*oracle_bits(ins), rows, causal=w.causal), rows, f"{w.name} split {nsplit}")
+
+
+def test_unit_count_overflow_is_refused_before_launch():
+    """2^30 heads split in two make 2^31 work units, more than the kernels count
+    in int: the call returns EINVAL without launching (the pointers are never
+    dereferenced, so placeholders serve)."""
+    import ctypes
+    from attention_kl_distillation_b200 import binding as B
+    lib = B.lib()
+    prob = B.problem(1, 1 << 30, 8, 512, 64, 64, False)
+    v = ctypes.c_void_p
+    ptrs = [v(1 << 20) for _ in range(7)]
+    before = lib.streamkl_launch_count()
+    st = lib.streamkl_fwd_splitk(ctypes.byref(prob), *ptrs, 2, v(1 << 20), ctypes.c_size_t(1 << 62), v(0))
+    assert st == B.EINVAL
+    assert lib.streamkl_launch_count() == before
