@@ -123,7 +123,10 @@ size_t streamkl_bwd_workspace_size(const streamkl_problem *prob);
  * upstream dL (fp32 [B][H][NQ]).  Outputs dQ1, dK1, dQ2, dK2 are bf16 with the
  * shapes of their inputs; any of them may be NULL, which skips it: dQ1 = dK1
  * = NULL is the page's configuration 1 (teacher P1 fixed), dQ2 = dK2 = NULL
- * its configuration 2 (student P2 fixed).  workspace must hold
+ * its configuration 2 (student P2 fixed).  With one side asked for, the fused
+ * algorithm runs a kernel specialised to it: only that side's dS is formed
+ * and contracted (for the teacher side without the student's exponential).
+ * workspace must hold
  * streamkl_bwd_workspace_size bytes of device memory, 256-byte aligned; its
  * contents on entry do not matter and on exit are unspecified.  Gradients are
  * not bitwise reproducible (fp32 atomics).
