@@ -163,6 +163,29 @@ def test_autograd_wrapper_matches_direct_call():
         assert err <= 1e-2   # fp32 atomics: not bitwise reproducible
 
 
+@pytest.mark.parametrize("frozen", ["teacher", "student"])
+def test_autograd_frozen_side_runs_one_sided(frozen):
+    """Distillation with a frozen side through the autograd wrapper: only the
+    trainable side gets gradients, equal to a direct one-sided call."""
+    from attention_kl_distillation_b200 import bwd, fwd, streamkl
+    from attention_kl_distillation_b200.inputs import make_inputs
+    w = workload(1, 2, 160, 300, 128, 128, True)
+    Q1, K1, Q2, K2 = cuda_inputs(make_inputs(w))
+    train = (False, False, True, True) if frozen == "teacher" else (True, True, False, False)
+    ins = [t.clone().requires_grad_(r) for t, r in zip((Q1, K1, Q2, K2), train)]
+    L = streamkl(*ins, causal=True)
+    L.sum().backward()
+    L0, A, B = fwd(Q1, K1, Q2, K2, causal=True)
+    ref = bwd(torch.ones_like(L0), Q1, K1, Q2, K2, L0, A, B, causal=True, need=train)
+    torch.cuda.synchronize()
+    for t, r, n in zip(ins, ref, train):
+        if not n:
+            assert t.grad is None and r is None
+            continue
+        err = ((t.grad.float() - r.float()).norm() / r.float().norm()).item()
+        assert err <= 1e-2   # fp32 atomics: not bitwise reproducible
+
+
 def test_bwd_full_size_workload(orc):
     """Forward+backward workload (B1 H32 N16384 d128 causal, dL = 1/(B*H*NQ)):
     dQ on >= 256 sampled rows of every head, dK1/dK2 in full on head 0 and one seeded head."""
