@@ -135,6 +135,25 @@ def profiled_traffic(profile: str):
     return int(m2.group(1))
 
 
+DATASHEET_BF16_TFLOPS = 2250.0  # dense (not 2:4 sparse) bf16 per GPU
+
+
+def peak_ratios(step_tf: float, fwd_tf: float, clk: dict, dev) -> dict:
+    """The per-GPU step and forward rates against three denominators: the dense bf16
+    datasheet figure, the measured cuBLAS figure, and the clock-normalised tensor peak
+    (SMs x 8192 FLOP/clk x the median SM clock sampled during the timed region)."""
+    peak, _, _ = peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = (clk or {}).get("sm_mhz")
+    clock_peak = sms * 8192 * mhz * 1e6 / 1e12 if mhz else None
+    out = {}
+    for name, v in (("step", step_tf), ("fwd", fwd_tf)):
+        out[name] = {"datasheet_dense_bf16": v / DATASHEET_BF16_TFLOPS, "measured_bf16": v / peak,
+                     "clock_normalised": (v / clock_peak) if clock_peak else None}
+    out["clock_peak_tflops"] = clock_peak
+    return out
+
+
 def step_flops(w: Workload, phase: str) -> int:
     return w.fwd_flops() + (w.bwd_flops() if phase == "fwdbwd" else 0)
 
@@ -219,6 +238,10 @@ def cpu_baseline(w: Workload, phase: str, target_s: float) -> dict:
         scale = (target_s / max(dt, 1e-3)) ** (0.5 if sub.NK == sub.NQ else 1.0)
         R = int(min(w.NQ, max(R, R * scale * 0.9)) // 64 * 64)
         dt, fl, sub = oracle_sample_run(w, phase, R, nthreads, w.seed)
+    pps = sub.visible_pairs() / dt
+    # one thread, on a smaller prefix (about a tenth of the threaded sample's time)
+    R1 = max(64, int(sub.NQ * (0.1 / nthreads) ** (0.5 if sub.NK == sub.NQ else 1.0)) // 64 * 64)
+    dt1, _, sub1 = oracle_sample_run(w, phase, min(R1, sub.NQ), 1, w.seed)
     return {
         "value": fl / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
         "seconds": dt,
@@ -226,6 +249,11 @@ def cpu_baseline(w: Workload, phase: str, target_s: float) -> dict:
                    f"{'causal' if sub.causal else 'non-causal'}) of the {w.name} recipe, "
                    f"{'forward+backward' if phase == 'fwdbwd' else 'forward'}; "
                    f"{fl / 1e9:.1f} GFLOP algorithmic"),
+        # rows are independent and the oracle's cost is linear in the visible pairs
+        "pairs_per_s": pps,
+        "full_config_s_extrapolated": w.visible_pairs() / pps,
+        "single_thread": {"pairs_per_s": sub1.visible_pairs() / dt1, "sample_rows": sub1.NQ,
+                          "seconds": dt1},
     }
 
 
@@ -464,6 +492,7 @@ def main(argv=None):
                    **({"splitk": nsplit} if nsplit else {}),
                    "parallelism": f"dp{world} (independent replicas, no collective)"},
         "pct_of_peak": value / world / peak,
+        "peak_ratios": peak_ratios(value / world, fwd_tf, clk, dev),
         "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac_of_peak": fwd_tf / peak,
                 "rows_per_s": w.BH * w.NQ / (fwd_ms * 1e-3)},
         "bwd": ({"ms": bwd_ms, "tflops": bwd_tf, "frac_of_peak": bwd_tf / peak}
