@@ -33,8 +33,10 @@
 //
 // Units are visited longest first (the last query tiles of a causal problem
 // see the most keys) and dealt to CTAs in a snake order, an approximation of
-// longest-processing-time scheduling; units of one query tile across heads
-// run together, so they stream the same key range through L2.
+// longest-processing-time scheduling.  When a head has at least one query tile
+// per SM, heads run one after another so that concurrent CTAs share its key
+// tiles in L2; otherwise the units of one query tile across all heads run
+// together.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -124,8 +126,17 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     w.split = u % p.nsplit;
     u /= p.nsplit;
   }
-  w.bh = u % p.BH;
-  w.q0 = (nqb - 1 - u / p.BH) * BQ;  // longest (last) query tiles first
+  // Heads in groups of p.head_group: within a group, query tiles longest first
+  // and heads innermost.  With one head per group, the CTAs running at one time
+  // all stream the same head's key tiles at about the same time, so long
+  // problems read K from L2 instead of HBM.  With every head in one group, the
+  // longest units of all heads come first, which keeps the last wave short.
+  const int G = max(1, min(p.head_group, p.BH));
+  const int g = u / (G * nqb);
+  const int gsize = min(G, p.BH - g * G);
+  const int r = u - g * G * nqb;
+  w.bh = g * G + r % gsize;
+  w.q0 = (nqb - 1 - r / gsize) * BQ;  // longest (last) query tiles first
   const int nkt_all = (p.NK + BK - 1) / BK;
   const int off = p.NK - p.NQ;
   w.kt_lo = p.nsplit > 1 ? w.split * p.kt_chunk : 0;

@@ -33,6 +33,9 @@ struct FwdParams {
   // ([nsplit][5][BH*NQ]: m1, m2, l1, l2, acc in the base-2 domain) instead of L/LSE.
   int kt_chunk, nsplit;
   float* part;
+  // Row-tile kernel: heads per group of the unit order (1 = heads one after
+  // another, BH = all heads interleaved per query tile).
+  int head_group;
 };
 
 struct FwdMergeParams {

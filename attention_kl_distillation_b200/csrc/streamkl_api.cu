@@ -319,6 +319,12 @@ streamkl_status prepare_fwd(const streamkl_problem* prob, const void* Q1, const 
   p->kt_chunk = 0;
   p->nsplit = 1;
   p->part = nullptr;
+  // One head at a time once a head has a query tile per SM: the concurrent CTAs
+  // then share its key tiles in L2 (B1 H32 N65536 causal: 52 -> 42 ms); smaller
+  // problems keep the order that interleaves all heads per query tile, whose
+  // last wave is shorter (N4096: 0.21 ms against 0.23).
+  const int nqt = (prob->NQ + skl::kFwdBQ - 1) / skl::kFwdBQ;
+  p->head_group = nqt >= dev->num_sms ? 1 : static_cast<int>(BH);
   *devp = dev;
   return STREAMKL_OK;
 }

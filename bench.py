@@ -60,6 +60,9 @@ def parse_args(argv=None):
                     help="override NQ (small-NQ forward cases; not a bench line)")
     ap.add_argument("--splitk", action="store_true",
                     help="run the forward through streamkl_fwd_splitk with the suggested split")
+    ap.add_argument("--table", action="store_true",
+                    help="instead of the bench line, one JSON line per recipe (median of >= 10 "
+                         "timed calls, >= 5 for long64k, after 3 warm-ups)")
     ap.add_argument("--need", default="1111",
                     help="which of dQ1 dK1 dQ2 dK2 the backward returns (e.g. 0101 = dK only)")
     return ap.parse_args(argv)
@@ -289,9 +292,55 @@ def run_reference(args, w: Workload, phase: str):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------- per-recipe table
+def run_table(args):
+    """Per recipe and phase: median CUDA-event time of the library calls, TFLOP/s, rows/s and
+    the fraction of the measured bf16 peak (the reporting the measurement plan asks for)."""
+    import attention_kl_distillation_b200 as skl
+    from attention_kl_distillation_b200 import binding
+    peak, _, _ = peaks()
+    dev = torch.device("cuda", 0)
+    for name in ("tiny", "causal4k", "sparse_student", "long64k", "fwdbwd16k"):
+        w = WORKLOADS[name]
+        Q1, K1, Q2, K2 = (t.to(dev) for t in make_inputs(w))
+        L, A, B = (torch.empty((w.B, w.H, w.NQ), device=dev) for _ in range(3))
+        dL = torch.full((w.B, w.H, w.NQ), 1.0 / (w.B * w.H * w.NQ), device=dev)
+        grads = tuple(torch.empty_like(t) for t in (Q1, K1, Q2, K2)) if w.backward else None
+        ws = (torch.empty(binding.workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal),
+                          dtype=torch.uint8, device=dev) if w.backward else None)
+        calls = [("fwd", lambda: skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B)), w.fwd_flops())]
+        if w.backward:
+            calls.append(("bwd", lambda: skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal,
+                                                 workspace=ws, out=grads), w.bwd_flops()))
+        n = 5 if name == "long64k" else 10
+        for phase, fn, fl in calls:
+            for _ in range(3):
+                fn()
+            times = []
+            for _ in range(n):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            ms = statistics.median(times)
+            tf = fl / (ms * 1e-3) / 1e12
+            print(json.dumps({"recipe": name, "phase": phase, "calls": n, "median_ms": ms,
+                              "tflops": tf, "frac_of_measured_bf16": tf / peak,
+                              "rows_per_s": w.BH * w.NQ / (ms * 1e-3),
+                              "mufu_ceiling_frac_of_clock_peak": (w.d1 + w.d2) / 512}), flush=True)
+        if skl.query_device_status() != 0:
+            raise RuntimeError("device status reported an error")
+        del Q1, K1, Q2, K2, L, A, B, dL, grads, ws
+        torch.cuda.empty_cache()
+
+
 # --------------------------------------------------------------------------- our path
 def main(argv=None):
     args = parse_args(argv)
+    if args.table:
+        return run_table(args)
     w = WORKLOADS[args.workload]
     if args.heads:
         w = w.with_(H=args.heads)
