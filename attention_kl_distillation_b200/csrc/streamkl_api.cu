@@ -397,7 +397,30 @@ int streamkl_fwd_splitk_suggest(const streamkl_problem* prob) {
   if (current_device(&dev) != STREAMKL_OK) return 0;
   const int units = fwd_unit_count(*prob, 1);
   const int sms = dev->num_sms;
-  if (units >= sms) return 1;
+  if (units >= sms) {
+    // Enough units already; without the causal mask they are all the same
+    // length, so a partly filled last wave idles SMs: split in two to four
+    // chunks when that fills the waves clearly better (B2 H16 NQ=2048
+    // NK=32768: 512 units are 3.46 waves, two chunks make 6.92).
+    if (prob->causal) return 1;
+    auto fill = [&](long long total) {
+      const long long waves = (total + sms - 1) / sms;
+      return static_cast<double>(total) / static_cast<double>(waves * sms);
+    };
+    int best = 1;
+    double best_fill = fill(units);
+    const int nkt = fwd_key_tiles(*prob);
+    for (int n = 2; n <= 4 && n <= nkt; ++n) {
+      int chunk, nsp;
+      split_shape(*prob, n, &chunk, &nsp);
+      const double f = fill(static_cast<long long>(units) * nsp);
+      if (f > best_fill + 0.05) {
+        best_fill = f;
+        best = nsp;
+      }
+    }
+    return best;
+  }
   // About four units per SM: measured on B200 for B1 H32 NK=32768 (32 and 64
   // unsplit units), fewer splits leave HBM idle in the last waves and more add
   // per-unit work (Q load, lane merge) and merge traffic.

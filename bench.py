@@ -309,6 +309,13 @@ def run_table(args):
         ws = (torch.empty(binding.workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal),
                           dtype=torch.uint8, device=dev) if w.backward else None)
         calls = [("fwd", lambda: skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B)), w.fwd_flops())]
+        ns = binding.splitk_suggest(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal)
+        if ns > 1 and name != "tiny":
+            fws = torch.empty(max(256, binding.splitk_workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, ns)),
+                              dtype=torch.uint8, device=dev)
+            calls.append((f"fwd_splitk{ns}",
+                          lambda: skl.fwd_splitk(Q1, K1, Q2, K2, causal=w.causal, nsplit=ns,
+                                                 workspace=fws, out=(L, A, B)), w.fwd_flops()))
         if w.backward:
             calls.append(("bwd", lambda: skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal,
                                                  workspace=ws, out=grads), w.bwd_flops()))
@@ -332,7 +339,7 @@ def run_table(args):
                               "mufu_ceiling_frac_of_clock_peak": (w.d1 + w.d2) / 512}), flush=True)
         if skl.query_device_status() != 0:
             raise RuntimeError("device status reported an error")
-        del Q1, K1, Q2, K2, L, A, B, dL, grads, ws
+        del Q1, K1, Q2, K2, L, A, B, dL, grads, ws, calls
         torch.cuda.empty_cache()
 
 

@@ -104,8 +104,11 @@ size_t streamkl_fwd_splitk_workspace_size(const streamkl_problem *prob, int nspl
 
 /*
  * A split count for the current device: about four of the forward's work
- * units per SM (at most one key tile per chunk); 1 when the problem already
- * has a unit per SM.  0 on a bad problem or if the device cannot be queried.
+ * units per SM (at most one key tile per chunk).  When the problem already
+ * has a unit per SM: 1 for a causal problem; otherwise the count from 1 to 4
+ * that fills the last wave of SMs clearly best (all units have the same
+ * length, so a partly filled last wave idles SMs).  0 on a bad problem or if
+ * the device cannot be queried.
  */
 int streamkl_fwd_splitk_suggest(const streamkl_problem *prob);
 
