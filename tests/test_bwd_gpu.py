@@ -208,3 +208,33 @@ def test_bwd_full_size_workload(orc):
     for n, G in (("dK1", dK1), ("dK2", dK2)):
         err = rel_frobenius(G.reshape(w.BH, w.NK, -1)[heads], o[n])
         assert err <= TOL_GRAD, f"{n} {err:.3e}"
+
+
+@pytest.mark.parametrize("side", ["student", "teacher"])
+def test_bwd_full_size_one_sided(orc, bwd_algo, side):
+    """The one-sided kernels on the forward+backward workload (B1 H32 N16384 d128
+    causal): the student side alone (the page's configuration 1, standard
+    distillation) or the teacher side alone; dQ on sampled rows of every head,
+    dK in full on head 0 and one seeded head.  The specialised kernels are the
+    fused path's; the split path is covered at this size by the test above."""
+    if bwd_algo != "fused":
+        pytest.skip("the one-sided kernels are the fused path")
+    from attention_kl_distillation_b200.inputs import WORKLOADS, make_inputs, sample_rows
+    w = WORKLOADS["fwdbwd16k"]
+    ins = make_inputs(w)
+    dev = cuda_inputs(ins)
+    g = 1.0 / (w.B * w.H * w.NQ)
+    dL = torch.full((w.B, w.H, w.NQ), g, device="cuda")
+    need = (False, False, True, True) if side == "student" else (True, True, False, False)
+    out = run_bwd(dev, dL, True, need=need)
+    dQ, dK = (out[2], out[3]) if side == "student" else (out[0], out[1])
+    assert all(out[i] is None for i in range(4) if not need[i])
+    bits = oracle_bits(ins)
+    rows = sample_rows(w.BH, w.NQ, 256, seed=w.seed + 1)
+    _, _, _, oq1, oq2 = orc.bwd_rows(*bits, rows, np.full(len(rows), g), causal=True)
+    gq = dQ.reshape(w.BH, w.NQ, -1)[rows[:, 0], rows[:, 1]]
+    assert rel_frobenius(gq, oq2 if side == "student" else oq1) <= TOL_GRAD
+    heads = [0, int(np.random.default_rng(w.seed + 1).integers(1, w.BH))]
+    o = orc.bwd_heads(*bits, heads, np.full((2, w.NQ), g), causal=True)
+    err = rel_frobenius(dK.reshape(w.BH, w.NK, -1)[heads], o["dK2" if side == "student" else "dK1"])
+    assert err <= TOL_GRAD, f"{side} dK {err:.3e}"
