@@ -102,3 +102,15 @@ def test_unit_count_overflow_is_refused_before_launch():
     st = lib.streamkl_fwd_splitk(ctypes.byref(prob), *ptrs, 2, v(1 << 20), ctypes.c_size_t(1 << 62), v(0))
     assert st == B.EINVAL
     assert lib.streamkl_launch_count() == before
+
+
+@pytest.mark.parametrize("nq", [1, 20])
+def test_transposed_unsplit_long_keys(orc, nq):
+    """The unsplit transposed forward on the 64K key set (B1 H32 NK=65536 causal):
+    one CTA streams all 512 key tiles of a head, every query row checked."""
+    from attention_kl_distillation_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS["long64k"].with_(NQ=nq)
+    ins = make_inputs(w)
+    gpu = gpu_fwd(cuda_inputs(ins), True)
+    rows = all_rows(w.BH, w.NQ)
+    check_fwd(gpu, orc.fwd_rows(*oracle_bits(ins), rows, causal=True), rows, f"long keys NQ={nq}")
