@@ -3,6 +3,7 @@
 The compute path is libstreamkl.so (sm_100a kernels behind a C ABI, see
 include/streamkl.h); ``streamkl`` is its thin Python binding.
 """
-from .binding import (StreamKLError, bwd, bwd_algorithm_for, fwd, fwd_splitk, launch_count,  # noqa: F401
-                      query_device_status, set_bwd_algorithm, set_wait_limit_ms, streamkl,
+from .binding import (StreamKLError, bwd, bwd_algorithm_for, bwd_noalloc, fwd,  # noqa: F401
+                      fwd_splitk, launch_count, query_device_status, set_bwd_algorithm,
+                      set_wait_limit_ms, splitk_suggest, splitk_workspace_size, streamkl,
                       workspace_size)
