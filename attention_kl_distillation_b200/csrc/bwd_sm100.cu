@@ -155,11 +155,11 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_
 #pragma unroll
     for (int h = 0; h < 2; ++h) {  // 4 queries per h
       const int q = c * 8 + h * 4;
-      const float4 nb1 = *reinterpret_cast<const float4*>(rr + 0 * BQ + q);
-      const float4 nb2 = *reinterpret_cast<const float4*>(rr + 1 * BQ + q);
-      const float4 nL = *reinterpret_cast<const float4*>(rr + 2 * BQ + q);
-      const float4 g1 = G1 ? *reinterpret_cast<const float4*>(rr + 3 * BQ + q) : float4{};
-      const float4 g2 = G2 ? *reinterpret_cast<const float4*>(rr + 4 * BQ + q) : float4{};
+      const float4 nb1 = ld_shared_f4(rr + 0 * BQ + q);
+      const float4 nb2 = ld_shared_f4(rr + 1 * BQ + q);
+      const float4 nL = ld_shared_f4(rr + 2 * BQ + q);
+      const float4 g1 = G1 ? ld_shared_f4(rr + 3 * BQ + q) : float4{};
+      const float4 g2 = G2 ? ld_shared_f4(rr + 4 * BQ + q) : float4{};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {  // a pair of queries
         const int i = q + 2 * e;

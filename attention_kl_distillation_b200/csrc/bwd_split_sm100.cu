@@ -141,11 +141,11 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[CPW], const uint32_
   for (int q = 0; q < CPW; q += 4) {
     float4 nb1, nb2, nL, g1, g2;
     if (COLREC) {
-      nb1 = *reinterpret_cast<const float4*>(rr + 0 * CB + q);
-      nb2 = *reinterpret_cast<const float4*>(rr + 1 * CB + q);
-      nL = *reinterpret_cast<const float4*>(rr + 2 * CB + q);
-      g1 = *reinterpret_cast<const float4*>(rr + 3 * CB + q);
-      g2 = *reinterpret_cast<const float4*>(rr + 4 * CB + q);
+      nb1 = ld_shared_f4(rr + 0 * CB + q);
+      nb2 = ld_shared_f4(rr + 1 * CB + q);
+      nL = ld_shared_f4(rr + 2 * CB + q);
+      g1 = ld_shared_f4(rr + 3 * CB + q);
+      g2 = ld_shared_f4(rr + 4 * CB + q);
     } else {
       nb1 = make_float4(rec[0], rec[0], rec[0], rec[0]);
       nb2 = make_float4(rec[1], rec[1], rec[1], rec[1]);

@@ -345,6 +345,18 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+// 16-byte load from shared memory by shared-space address.  The kernels read
+// per-query records that every lane of a warp needs at the same address;
+// through a generic pointer such loads took several shared-memory wavefronts
+// each, as a shared-space load they are one broadcast.
+__device__ __forceinline__ float4 ld_shared_f4(const void* p) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
+
 // Named barrier among `nthreads` threads (multiple of 32).
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
