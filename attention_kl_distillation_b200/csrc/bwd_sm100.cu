@@ -139,15 +139,19 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // dS for one key row and QPW queries of a step (pairs of queries at a time,
 // packed f32x2).  s1/s2: raw products <K_t[key], Q_t[q]> from TMEM; rr: the
 // step's field-major row records offset to this half; w1/w2 receive the bf16
-// pairs of s1*dS1^T and s2*dS2^T for these queries.
+// pairs of s1*dS1^T and s2*dS2^T for these queries.  EARLY: also store each
+// 8-query chunk into row j of the dS tiles as soon as it is formed, so that
+// the stores overlap the arithmetic (the buffer must already be free).
 //   u_t = log2 P_t = c_t S_t - LSE_t log2e
 //   dS1 = s1 dL P1 (ln2 (u1 - u2) - L),   dS2 = s2 dL (P2 - P1)
 // MASK: visible iff key < NK and (not causal or q >= thr), with thr the first
 // visible query index of this half for this key.
-template <bool MASK, bool G1, bool G2>
+template <bool MASK, bool G1, bool G2, bool EARLY = false>
 __device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_t (&s2)[QPW],
                                         const float* rr, float c1, float c2, bool key_ok, int thr,
-                                        uint32_t (&w1)[QPW / 2], uint32_t (&w2)[QPW / 2]) {
+                                        uint32_t (&w1)[QPW / 2], uint32_t (&w2)[QPW / 2],
+                                        int j = 0, int c0 = 0, uint32_t ds1_row = 0,
+                                        uint32_t ds2_row = 0) {
   const float2 C1 = make_float2(c1, c1), C2 = make_float2(c2, c2);
   const float2 NEG1 = make_float2(-1.f, -1.f), LN2 = make_float2(kLn2, kLn2);
 #pragma unroll
@@ -192,6 +196,11 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[QPW], const uint32_
         if (G1) w1[c * 4 + h * 2 + e] = pack_bf16(d1.x, d1.y);
         if (G2) w2[c * 4 + h * 2 + e] = pack_bf16(d2.x, d2.y);
       }
+    }
+    if (EARLY) {  // this 8-query chunk goes to shared memory at once (swizzle as in store_ds)
+      const uint32_t sw = static_cast<uint32_t>(((c0 + c) ^ (j & 7)) << 4);
+      if (G1) st_shared_v4(ds1_row + sw, w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
+      if (G2) st_shared_v4(ds2_row + sw, w2[4 * c], w2[4 * c + 1], w2[4 * c + 2], w2[4 * c + 3]);
     }
   }
 }
@@ -534,18 +543,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         const float* rr = rr_s(qs) + part * QPW;
         const bool masked = (p.causal && q0 + off < w.k0 + BK - 1) || (w.k0 + BK > p.NK);
         uint32_t w1[QPW / 2], w2[QPW / 2];
-        if (masked) {
-          // first visible query (index within this half) for this key
-          const int thr = p.causal ? key - off - q0 - part * QPW : -1;
-          form_ds<true, G1, G2>(a, b, rr, p.c1, p.c2, key_ok, thr, w1, w2);
+        const int thr = p.causal ? key - off - q0 - part * QPW : -1;  // first visible query
+        const uint32_t r1 = smem_u32(ds1_s(db)) + j * 128, r2 = smem_u32(ds2_s(db)) + j * 128;
+        if (DSB >= 2) {
+          // With two dS buffers the one this step writes was freed a step ago:
+          // wait for it first and store as the chunks are formed.
+          if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
+          dsph[db] ^= 1;
+          if (masked)
+            form_ds<true, G1, G2, true>(a, b, rr, p.c1, p.c2, key_ok, thr, w1, w2, j,
+                                        part * (QPW / 8), r1, r2);
+          else
+            form_ds<false, G1, G2, true>(a, b, rr, p.c1, p.c2, true, 0, w1, w2, j,
+                                         part * (QPW / 8), r1, r2);
         } else {
-          form_ds<false, G1, G2>(a, b, rr, p.c1, p.c2, true, 0, w1, w2);
+          // One buffer: form dS in registers while the previous step's
+          // contractions still read it.
+          if (masked)
+            form_ds<true, G1, G2>(a, b, rr, p.c1, p.c2, key_ok, thr, w1, w2);
+          else
+            form_ds<false, G1, G2>(a, b, rr, p.c1, p.c2, true, 0, w1, w2);
+          // the buffer is free once the contractions of the step that used it are done
+          if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
+          dsph[db] ^= 1;
+          store_ds<G1, G2>(w1, w2, j, part * (QPW / 8), r1, r2);
         }
-        // the buffer is free once the contractions of the step that used it are done
-        if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
-        dsph[db] ^= 1;
-        store_ds<G1, G2>(w1, w2, j, part * (QPW / 8), smem_u32(ds1_s(db)) + j * 128,
-                 smem_u32(ds2_s(db)) + j * 128);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&dsfull[db]);
