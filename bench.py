@@ -319,6 +319,15 @@ def run_table(args):
         if w.backward:
             calls.append(("bwd", lambda: skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal,
                                                  workspace=ws, out=grads), w.bwd_flops()))
+            # one gradient side (teacher fixed: dQ2, dK2; student fixed: dQ1, dK1): both S
+            # products are recomputed, the contractions of the other side are not done
+            pairs = w.bwd_flops() / (6 * (w.d1 + w.d2))
+            for side, keep, d in (("student", (2, 3), w.d2), ("teacher", (0, 1), w.d1)):
+                outs = tuple(g if i in keep else None for i, g in enumerate(grads))
+                calls.append((f"bwd_{side}_side",
+                              lambda outs=outs: skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal,
+                                                        workspace=ws, out=outs),
+                              pairs * (2 * (w.d1 + w.d2) + 4 * d)))
         n = 5 if name == "long64k" else 10
         for phase, fn, fl in calls:
             for _ in range(3):
