@@ -50,6 +50,8 @@ _lib.streamkl_bwd.argtypes = [_pp] + [_vp] * 13 + [ctypes.c_size_t, _vp]
 _lib.streamkl_bwd.restype = ctypes.c_int
 _lib.streamkl_bwd_noalloc.argtypes = [_pp] + [_vp] * 13
 _lib.streamkl_bwd_noalloc.restype = ctypes.c_int
+_lib.streamkl_bwd_noalloc_scratch_bytes.argtypes = []
+_lib.streamkl_bwd_noalloc_scratch_bytes.restype = ctypes.c_size_t
 _lib.streamkl_status_string.argtypes = [ctypes.c_int]
 _lib.streamkl_status_string.restype = ctypes.c_char_p
 _lib.streamkl_query_device_status.argtypes = [_vp]
@@ -134,9 +136,9 @@ def _ptr(t):
     return _vp(t.data_ptr()) if t is not None else _vp(0)
 
 
-def _check_qk(Q1, K1, Q2, K2):
+def _check_qk(Q1, K1, Q2, K2, require_cuda=True):
     for n, t in (("Q1", Q1), ("K1", K1), ("Q2", Q2), ("K2", K2)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 4 or not t.is_contiguous():
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
             raise ValueError(f"{n} must be a contiguous CUDA bf16 tensor [B, H, N, d]")
     B, H, NQ, d1 = Q1.shape
     NK = K1.shape[2]
@@ -145,7 +147,35 @@ def _check_qk(Q1, K1, Q2, K2):
         raise ValueError("inconsistent shapes of Q1, K1, Q2, K2")
     if len({Q1.device, K1.device, Q2.device, K2.device}) != 1:
         raise ValueError("inputs must be on one device")
+    if require_cuda and not Q1.is_cuda:
+        raise ValueError("inputs must be CUDA tensors")
     return B, H, NQ, NK, d1, d2
+
+
+def _check_bwd(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, out, require_cuda=True):
+    """Checks every tensor the backward entry points receive; the library sees only raw
+    pointers, so a wrong dtype, shape, layout or device must be refused here.  `out`
+    holds the four gradient tensors or None entries (None skips that gradient)."""
+    dims = _check_qk(Q1, K1, Q2, K2, require_cuda=False)
+    B, H, NQ = dims[:3]
+    for n, t in (("dL", dL), ("L", L), ("LSE1", LSE1), ("LSE2", LSE2)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or t.shape != (B, H, NQ) \
+                or not t.is_contiguous() or t.device != Q1.device:
+            raise ValueError(f"{n} must be a contiguous fp32 tensor [B, H, NQ] on the inputs' device")
+    if out is not None:
+        if len(out) != 4:
+            raise ValueError("out must hold four entries: dQ1, dK1, dQ2, dK2 (None skips one)")
+        for n, o, t in zip(("dQ1", "dK1", "dQ2", "dK2"), out, (Q1, K1, Q2, K2)):
+            if o is not None and (not isinstance(o, torch.Tensor) or o.shape != t.shape
+                                  or o.dtype != torch.bfloat16 or not o.is_contiguous()
+                                  or o.device != t.device):
+                raise ValueError(f"gradient output {n} must match its input "
+                                 f"(bf16, contiguous, shape {tuple(t.shape)}, same device)")
+        if all(o is None for o in out):
+            raise ValueError("out asks for no gradient")
+    if require_cuda and not Q1.is_cuda:
+        raise ValueError("inputs must be CUDA tensors")
+    return dims
 
 
 def _stream(device):
@@ -220,18 +250,10 @@ def bwd(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, causal=False, s1=None, s2=None,
 
     ``out`` may pass preallocated gradient tensors (None entries are skipped);
     ``workspace`` a preallocated device buffer of at least ``workspace_size`` bytes."""
-    B, H, NQ, NK, d1, d2 = _check_qk(Q1, K1, Q2, K2)
-    for n, t in (("dL", dL), ("L", L), ("LSE1", LSE1), ("LSE2", LSE2)):
-        if t.dtype != torch.float32 or t.shape != (B, H, NQ) or not t.is_contiguous() \
-                or t.device != Q1.device:
-            raise ValueError(f"{n} must be a contiguous fp32 tensor [B, H, NQ] on the inputs' device")
+    B, H, NQ, NK, d1, d2 = _check_bwd(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, out)
     prob = problem(B, H, NQ, NK, d1, d2, causal, s1, s2)
     if out is not None:
         outs = list(out)
-        for o, t in zip(outs, (Q1, K1, Q2, K2)):
-            if o is not None and (o.shape != t.shape or o.dtype != torch.bfloat16
-                                  or not o.is_contiguous() or o.device != t.device):
-                raise ValueError("gradient outputs must match their inputs (bf16, contiguous)")
     else:
         outs = [torch.empty_like(t) if want else None
                 for t, want in zip((Q1, K1, Q2, K2), need)]
@@ -251,14 +273,18 @@ def bwd(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, causal=False, s1=None, s2=None,
     return tuple(outs)
 
 
-NOALLOC_SCRATCH_BYTES = 64 << 20
+# Size of the static device scratch streamkl_bwd_noalloc uses, as the library reports it.
+NOALLOC_SCRATCH_BYTES = int(_lib.streamkl_bwd_noalloc_scratch_bytes())
 
 
 def bwd_noalloc(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, out, causal=False, s1=None, s2=None):
     """streamkl_bwd_noalloc: the backward without a caller workspace, for callers that
-    cannot allocate device memory.  ``out`` holds preallocated bf16 gradients (None skips
-    one); the library's own static scratch (64 MiB per GPU) replaces the workspace."""
-    B, H, NQ, NK, d1, d2 = _check_qk(Q1, K1, Q2, K2)
+    cannot allocate device memory.  ``out`` holds four preallocated bf16 gradients (None
+    skips one); the library's own static scratch (NOALLOC_SCRATCH_BYTES per GPU) replaces
+    the workspace.  Every tensor is checked as in ``bwd`` before the call."""
+    if out is None:
+        raise ValueError("bwd_noalloc needs preallocated gradient outputs")
+    B, H, NQ, NK, d1, d2 = _check_bwd(dL, Q1, K1, Q2, K2, L, LSE1, LSE2, out)
     prob = problem(B, H, NQ, NK, d1, d2, causal, s1, s2)
     with torch.cuda.device(Q1.device):
         st = _lib.streamkl_bwd_noalloc(ctypes.byref(prob), _ptr(dL), _ptr(Q1), _ptr(K1), _ptr(Q2),

@@ -36,7 +36,9 @@ struct DeviceInfo {
 
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
-unsigned long long g_wait_limit_ns = 0;
+// Settings any host thread may change while others launch: atomics, written by
+// the setters and initialised once from the environment on first read.
+std::atomic<unsigned long long> g_wait_limit_ns{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -45,15 +47,19 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 EncodeTiledFn g_encode = nullptr;
 
 unsigned long long wait_limit_ns() {
-  if (g_wait_limit_ns == 0) {
+  unsigned long long v = g_wait_limit_ns.load();
+  if (v == 0) {
     long ms = 2000;
     if (const char* e = std::getenv("STREAMKL_WAIT_LIMIT_MS")) {
-      long v = std::strtol(e, nullptr, 10);
-      if (v >= 1) ms = v;
+      long x = std::strtol(e, nullptr, 10);
+      if (x >= 1) ms = x;
     }
-    g_wait_limit_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+    unsigned long long expect = 0;
+    // a concurrent streamkl_set_wait_limit_ms wins over the environment default
+    g_wait_limit_ns.compare_exchange_strong(expect, static_cast<unsigned long long>(ms) * 1000000ull);
+    v = g_wait_limit_ns.load();
   }
-  return g_wait_limit_ns;
+  return v;
 }
 
 // Device of the current thread, probed once: sm_100 check, SM count, status word.
@@ -169,18 +175,22 @@ struct BwdWorkspace {
 };
 
 // Backward algorithm: process-wide setting, environment default read once.
-int g_bwd_algo = -1;
+std::atomic<int> g_bwd_algo{-1};
 
 int bwd_algo_setting() {
-  if (g_bwd_algo < 0) {
+  int v = g_bwd_algo.load();
+  if (v < 0) {
     int a = STREAMKL_BWD_AUTO;
     if (const char* e = std::getenv("STREAMKL_BWD_ALGO")) {
       if (!std::strcmp(e, "fused")) a = STREAMKL_BWD_FUSED;
       else if (!std::strcmp(e, "split")) a = STREAMKL_BWD_SPLIT;
     }
-    g_bwd_algo = a;
+    int expect = -1;
+    // a concurrent streamkl_set_bwd_algorithm wins over the environment default
+    g_bwd_algo.compare_exchange_strong(expect, a);
+    v = g_bwd_algo.load();
   }
-  return g_bwd_algo;
+  return v;
 }
 
 // AUTO: the page keeps the fused kernel while its dQ reductions stay cheap and
@@ -241,7 +251,7 @@ streamkl_status streamkl_debug_inject(int mode) {
 streamkl_status streamkl_set_bwd_algorithm(streamkl_bwd_algorithm algo) {
   if (algo != STREAMKL_BWD_AUTO && algo != STREAMKL_BWD_FUSED && algo != STREAMKL_BWD_SPLIT)
     return STREAMKL_EINVAL;
-  g_bwd_algo = algo;
+  g_bwd_algo.store(algo);
   return STREAMKL_OK;
 }
 
@@ -252,7 +262,7 @@ streamkl_bwd_algorithm streamkl_bwd_algorithm_for(const streamkl_problem* prob) 
 
 streamkl_status streamkl_set_wait_limit_ms(int ms) {
   if (ms < 1) return STREAMKL_EINVAL;
-  g_wait_limit_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+  g_wait_limit_ns.store(static_cast<unsigned long long>(ms) * 1000000ull);
   return STREAMKL_OK;
 }
 

@@ -6,8 +6,9 @@
 // must not call cudaMalloc/cudaFree because those calls may synchronise the
 // whole device.  streamkl_bwd already allocates nothing, but it asks the
 // caller for a workspace.  streamkl_bwd_noalloc instead uses scratch that
-// this library owns: one statically sized device array, reserved on every
-// GPU that loads the library and kept until the process exits.
+// this library owns: one statically sized device array, reserved on a GPU
+// when this module is loaded there (at context creation under eager module
+// loading, at first use under lazy loading) and kept until the process exits.
 #include "streamkl.h"
 
 #include <cuda_runtime.h>
@@ -55,4 +56,8 @@ extern "C" streamkl_status streamkl_bwd_noalloc(const streamkl_problem* prob, co
   // (the dQ accumulator and the work-unit counter) on every call.
   return streamkl_bwd(prob, dL, Q1, K1, Q2, K2, L, LSE1, LSE2, dQ1, dK1, dQ2, dK2, scratch,
                       STREAMKL_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" size_t streamkl_bwd_noalloc_scratch_bytes(void) {
+  return STREAMKL_NOALLOC_SCRATCH_BYTES;
 }

@@ -9,8 +9,9 @@ d1=d2=128 causal with dL = 1/(B*H*NQ).  Inputs (537 MB) are larger than the
 
 Prints one JSON line (rank 0).  With torchrun (N > 1) every rank runs an
 independent replica of the workload (weak scaling: the path has no data
-exchange); the timed region is bracketed by barriers and the max over ranks
-is taken.
+exchange), or with ``--shard heads`` a contiguous range of the workload's
+B*H heads (strong scaling: the heads are independent problems); the timed
+region is bracketed by barriers and the max over ranks is taken.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores on a
 bounded sample of the same workload (the only other place this file runs the
@@ -63,6 +64,9 @@ def parse_args(argv=None):
     ap.add_argument("--table", action="store_true",
                     help="instead of the bench line, one JSON line per recipe (median of >= 10 "
                          "timed calls, >= 5 for long64k, after 3 warm-ups)")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: every rank runs the whole workload (replicas, weak scaling) or "
+                         "a contiguous range of its B*H heads (heads, strong scaling)")
     ap.add_argument("--need", default="1111",
                     help="which of dQ1 dK1 dQ2 dK2 the backward returns (e.g. 0101 = dK only)")
     return ap.parse_args(argv)
@@ -97,6 +101,16 @@ def workload_desc(w: Workload, phase: str) -> dict:
               + ("no flush (inputs larger than L2)" if w.input_bytes() > 126e6
                  else "L2 flushed between steps"),
     }
+
+
+def run_config(args, w: Workload, phase: str, world: int, nsplit=None) -> dict:
+    """The `config` object of a bench line; the reference arm prints the same one."""
+    if args.shard == "heads":
+        par = f"heads{world} (contiguous ranges of the B*H heads per GPU, no collective)"
+    else:
+        par = f"dp{world} (independent replicas, no collective)"
+    return {**workload_desc(w, phase), **({"need": args.need} if args.need != "1111" else {}),
+            **({"splitk": nsplit} if nsplit else {}), "parallelism": par}
 
 
 # The sources a profiled kernel is built from: its own file and the two shared headers.
@@ -282,7 +296,7 @@ def run_reference(args, w: Workload, phase: str):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "impl": "reference", "config": workload_desc(w, phase),
+        "data": "synthetic", "impl": "reference", "config": run_config(args, w, phase, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
                          "sample": f"first {sub.NQ} query rows of one head per step "
                                    f"({sub.NK} keys), {fl / 1e9:.1f} GFLOP algorithmic"},
@@ -383,9 +397,19 @@ def main(argv=None):
     from attention_kl_distillation_b200.parallel import max_over_ranks
 
     dev = torch.device("cuda", local)
-    cpu_ins = make_inputs(w, seed=w.seed + rank)  # independent replica per rank
+    full_w = w
+    if args.shard == "heads":
+        # strong scaling: this rank's contiguous range of the B*H heads, as a B = 1 problem
+        from attention_kl_distillation_b200.parallel import head_shard, shard_heads
+        if world > w.BH:
+            raise SystemExit(f"--shard heads needs at most {w.BH} ranks")
+        a, b = head_shard(w.BH, world, rank)
+        cpu_ins = [shard_heads(t, world, rank) for t in make_inputs(w)]
+        w = w.with_(B=1, H=b - a)
+    else:
+        cpu_ins = make_inputs(w, seed=w.seed + rank)  # independent replica per rank
     Q1, K1, Q2, K2 = (t.to(dev) for t in cpu_ins)
-    g = 1.0 / (w.B * w.H * w.NQ)
+    g = 1.0 / (full_w.B * full_w.H * full_w.NQ)  # the mean over the whole job's rows
     dL = torch.full((w.B, w.H, w.NQ), g, device=dev)
     L, A, B = (torch.empty((w.B, w.H, w.NQ), device=dev) for _ in range(3))
     need = tuple(c == "1" for c in args.need)
@@ -450,11 +474,13 @@ def main(argv=None):
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) if phase == "fwdbwd" else 0.0
     fl_step = step_flops(w, phase)
-    value = world * fl_step * args.steps / (total_ms * 1e-3) / 1e12
+    # whole-job work per step: every rank's replica, or the whole workload once when sharded
+    job_fl_step = step_flops(full_w, phase) if args.shard == "heads" else world * fl_step
+    value = job_fl_step * args.steps / (total_ms * 1e-3) / 1e12
     peak, hbm, src = peaks()
     fwd_tf = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
     bwd_tf = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if bwd_ms > 0 else None
-    full_size = w == WORKLOADS[args.workload] and args.need == "1111"
+    full_size = w == WORKLOADS[args.workload] and args.need == "1111" and not args.heads
     algo = binding.bwd_algorithm_for(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal)
     if phase == "fwdbwd" and bwd_ms >= fwd_ms:
         dom = {"kernel": f"streamkl_bwd, {algo} (prep + main + convert kernels)",
@@ -535,14 +561,14 @@ def main(argv=None):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
-        e2e = {"value": world * fl_step * ke / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_fl_step * ke / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / ke, "api": "attention_kl_distillation_b200.streamkl",
                "pipeline": "inputs of step k+1 copied on a side stream during step k (step 0's copy is not overlapped); result L read back every step"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, phase, args.cpu_seconds)
+        cpu = cpu_baseline(full_w, phase, args.cpu_seconds)
 
     if dist is not None:
         dist.destroy_process_group()
@@ -551,13 +577,14 @@ def main(argv=None):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
+        "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) teacher, student = teacher + noise; bf16)",
-        "config": {**workload_desc(w, phase), **({"need": args.need} if args.need != "1111" else {}),
-                   **({"splitk": nsplit} if nsplit else {}),
-                   "parallelism": f"dp{world} (independent replicas, no collective)"},
+        "config": run_config(args, full_w, phase, world, nsplit),
         "pct_of_peak": value / world / peak,
         "peak_ratios": peak_ratios(value / world, fwd_tf, clk, dev),
+        **({"heads_per_rank": [head_shard(full_w.BH, world, r)[1] - head_shard(full_w.BH, world, r)[0]
+                               for r in range(world)]} if args.shard == "heads" else {}),
         "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac_of_peak": fwd_tf / peak,
                 "rows_per_s": w.BH * w.NQ / (fwd_ms * 1e-3)},
         "bwd": ({"ms": bwd_ms, "tflops": bwd_tf, "frac_of_peak": bwd_tf / peak}

@@ -142,10 +142,19 @@ streamkl_status streamkl_bwd(const streamkl_problem *prob, const float *dL, cons
                              void *dK2, void *workspace, size_t ws_bytes, streamkl_stream_t stream);
 
 /*
- * Device scratch owned by streamkl_bwd_noalloc: 64 MiB, reserved on every GPU
- * that loads this library and held until the process exits.
+ * Device scratch owned by streamkl_bwd_noalloc: 64 MiB per GPU.  It is a
+ * static device array of the library's module, so it is reserved on a GPU
+ * when the module is loaded there and held until the process exits.  With
+ * eager module loading that happens at context creation; under CUDA's lazy
+ * loading (the default since CUDA 12.2, CUDA_MODULE_LOADING=LAZY) it happens
+ * at the module's first use on that GPU, which is the first
+ * streamkl_bwd_noalloc call (its address lookup) or the first launch of any
+ * of the library's kernels there.
  */
 #define STREAMKL_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* STREAMKL_NOALLOC_SCRATCH_BYTES as the built library has it (no CUDA call). */
+size_t streamkl_bwd_noalloc_scratch_bytes(void);
 
 /*
  * Backward for callers that cannot allocate device memory (the paper has no
@@ -159,8 +168,10 @@ streamkl_status streamkl_bwd(const streamkl_problem *prob, const float *dL, cons
  *    STREAMKL_NOALLOC_SCRATCH_BYTES are rejected with STREAMKL_EINVAL before
  *    any CUDA call.
  *  - The first call on a device looks up the scratch's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress) with that device current; under lazy module
+ *    loading that lookup is also what loads the module and reserves the
+ *    scratch on that device.  Make that first call before any stream
+ *    capture.
  *  - Every call on a device shares the one scratch array, which keeps the
  *    last call's contents (each call clears what must start at zero).  Calls
  *    that overlap on the GPU (different streams, or threads without ordering)

@@ -34,6 +34,27 @@ def test_reference_arm_prints_one_contract_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"].startswith("tiny")
+    # the same config keys as the GPU arm's line
+    assert set(line["config"]) == set(bench_config_keys())
+
+
+def bench_config_keys():
+    import bench
+    from attention_kl_distillation_b200.inputs import WORKLOADS
+    return bench.run_config(bench.parse_args([]), WORKLOADS["tiny"], "fwd", 1).keys()
+
+
+def test_reference_arm_does_not_load_the_library():
+    """The reference arm runs only the oracle: the CUDA library must not be mapped."""
+    code = ("import sys; sys.argv = ['bench.py']; import bench; "
+            "bench.main(['--impl', 'reference', '--workload', 'tiny', '--steps', '1', "
+            "'--warmup', '0']); "
+            "maps = open('/proc/self/maps').read(); "
+            "assert 'libstreamkl' not in maps, 'libstreamkl.so mapped'; "
+            "assert 'liboracle' in maps")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
 
 
 def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
@@ -60,6 +81,7 @@ def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
 @pytest.mark.parametrize("argv,expect", [
     ([], {"gpus": 1, "steps": 40, "warmup": 5, "impl": "ours", "workload": "fwdbwd16k"}),
     (["--nq", "1", "--splitk", "--phase", "fwd"], {"nq": 1, "splitk": True, "phase": "fwd"}),
+    (["--shard", "heads"], {"shard": "heads"}),
 ])
 def test_bench_arguments(argv, expect):
     import bench

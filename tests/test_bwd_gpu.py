@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_common import TOL_GRAD, cuda_inputs, oracle_bits, rel_frobenius, workload
+from gpu_common import TOL_GRAD, check_fwd, cuda_inputs, oracle_bits, rel_frobenius, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -28,13 +28,19 @@ SHAPES = [  # B, H, NQ, NK, d1, d2, causal
 ]
 
 
-def run_bwd(dev, dL, causal, need=(True, True, True, True), s1=None, s2=None):
+def run_bwd(dev, dL, causal, need=(True, True, True, True), s1=None, s2=None, saved=False):
+    """Forward then backward through the C ABI.  With saved=True also returns the
+    forward's L, LSE1, LSE2 ([BH, NQ] float64), the state the backward consumed."""
     from attention_kl_distillation_b200 import bwd, fwd, query_device_status
     L, A, B = fwd(*dev, causal=causal, s1=s1, s2=s2)
     grads = bwd(dL, *dev, L, A, B, causal=causal, s1=s1, s2=s2, need=need)
     torch.cuda.synchronize()
     assert query_device_status() == 0
-    return [g.float().cpu().numpy().astype(np.float64) if g is not None else None for g in grads]
+    out = [g.float().cpu().numpy().astype(np.float64) if g is not None else None for g in grads]
+    if saved:
+        BH = L.shape[0] * L.shape[1]
+        return out, tuple(t.reshape(BH, -1).cpu().numpy().astype(np.float64) for t in (L, A, B))
+    return out
 
 
 def oracle_heads(orc, ins, dL, causal, heads, s1=None, s2=None):
@@ -188,17 +194,20 @@ def test_autograd_frozen_side_runs_one_sided(frozen):
 
 def test_bwd_full_size_workload(orc):
     """Forward+backward workload (B1 H32 N16384 d128 causal, dL = 1/(B*H*NQ)):
-    dQ on >= 256 sampled rows of every head, dK1/dK2 in full on head 0 and one seeded head."""
+    the forward's L, LSE1, LSE2 and dQ on >= 256 sampled rows of every head,
+    dK1/dK2 in full on head 0 and one seeded head."""
     from attention_kl_distillation_b200.inputs import WORKLOADS, make_inputs, sample_rows
     w = WORKLOADS["fwdbwd16k"]
     ins = make_inputs(w)
     dev = cuda_inputs(ins)
     g = 1.0 / (w.B * w.H * w.NQ)
     dL = torch.full((w.B, w.H, w.NQ), g, device="cuda")
-    dQ1, dK1, dQ2, dK2 = run_bwd(dev, dL, True)
+    (dQ1, dK1, dQ2, dK2), fwd_out = run_bwd(dev, dL, True, saved=True)
     bits = oracle_bits(ins)
     rows = sample_rows(w.BH, w.NQ, 256, seed=w.seed)
-    _, _, _, oq1, oq2 = orc.bwd_rows(*bits, rows, np.full(len(rows), g), causal=True)
+    oL, oA, oB, oq1, oq2 = orc.bwd_rows(*bits, rows, np.full(len(rows), g), causal=True)
+    # the saved state the backward consumed: L, LSE1, LSE2 of the same rows
+    check_fwd(fwd_out, (oL, oA, oB), rows, "fwdbwd16k forward")
     gq1 = dQ1.reshape(w.BH, w.NQ, -1)[rows[:, 0], rows[:, 1]]
     gq2 = dQ2.reshape(w.BH, w.NQ, -1)[rows[:, 0], rows[:, 1]]
     assert rel_frobenius(gq1, oq1) <= TOL_GRAD
@@ -208,6 +217,10 @@ def test_bwd_full_size_workload(orc):
     for n, G in (("dK1", dK1), ("dK2", dK2)):
         err = rel_frobenius(G.reshape(w.BH, w.NK, -1)[heads], o[n])
         assert err <= TOL_GRAD, f"{n} {err:.3e}"
+    # every row of those two heads: the forward's saved state against the oracle's
+    hrows = np.stack(np.meshgrid(heads, np.arange(w.NQ), indexing="ij"), -1).reshape(-1, 2)
+    check_fwd(fwd_out, (o["L"].ravel(), o["LSE1"].ravel(), o["LSE2"].ravel()), hrows,
+              "fwdbwd16k forward, whole heads")
 
 
 @pytest.mark.parametrize("side", ["student", "teacher"])

@@ -90,7 +90,7 @@ def test_fwd_key_permutation_invariance():
     assert np.abs(A - Ap).max() <= 1e-5 and np.abs(B - Bp).max() <= 1e-5
 
 
-@pytest.mark.parametrize("name", ["causal4k", "sparse_student", "long64k"])
+@pytest.mark.parametrize("name", ["causal4k", "sparse_student", "long64k", "fwdbwd16k"])
 def test_fwd_full_size_sampled(orc, name):
     """Full-size workloads, >= 256 seeded rows per head plus the tile/causal edge rows."""
     from attention_kl_distillation_b200.inputs import WORKLOADS, make_inputs, sample_rows

@@ -24,6 +24,49 @@ def test_noalloc_rejects_problem_larger_than_scratch():
     assert B.lib().streamkl_bwd_noalloc(ctypes.byref(prob), *ptrs, ctypes.c_void_p(0)) == B.EINVAL
 
 
+def _cpu_args(NQ=40, NK=48, d1=64, d2=64):
+    g = torch.Generator().manual_seed(5)
+    Q1, K1, Q2, K2 = (torch.randn(1, 2, n, d, generator=g).to(torch.bfloat16)
+                      for n, d in ((NQ, d1), (NK, d1), (NQ, d2), (NK, d2)))
+    vec = [torch.zeros(1, 2, NQ) for _ in range(4)]     # dL, L, LSE1, LSE2
+    out = [torch.empty_like(t) for t in (Q1, K1, Q2, K2)]
+    return [vec[0], Q1, K1, Q2, K2, *vec[1:]], out
+
+
+@pytest.mark.parametrize("case", ["short_out", "wrong_shape", "wrong_dtype", "strided",
+                                  "bf16_dL", "wrong_L_shape", "no_output"])
+def test_noalloc_refuses_bad_tensors_before_any_call(case):
+    """The library receives raw pointers only, so the binding refuses anything that
+    would make the kernels read or write out of bounds, on the host, before a call."""
+    args, out = _cpu_args()
+    if case == "short_out":
+        out = out[:3]
+    elif case == "wrong_shape":
+        out[1] = torch.empty(1, 2, 47, 64, dtype=torch.bfloat16)
+    elif case == "wrong_dtype":
+        out[0] = out[0].float()
+    elif case == "strided":
+        out[2] = torch.empty(1, 2, 64, 40, dtype=torch.bfloat16).transpose(2, 3)
+    elif case == "bf16_dL":
+        args[0] = args[0].to(torch.bfloat16)
+    elif case == "wrong_L_shape":
+        args[5] = torch.zeros(1, 2, 41)
+    elif case == "no_output":
+        out = [None] * 4
+    calls = B.launch_count()
+    with pytest.raises(ValueError):
+        B.bwd_noalloc(*args, out)
+    assert B.launch_count() == calls
+
+
+def test_noalloc_scratch_size_matches_header():
+    import re
+    text = B.HEADER.read_text()
+    m = re.search(r"#define STREAMKL_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m, "macro not found in the header"
+    assert B.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point():
     from gpu_common import TOL_GRAD, cuda_inputs, rel_frobenius, workload
