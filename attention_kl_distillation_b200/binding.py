@@ -93,11 +93,12 @@ def launch_count() -> int:
     return int(_lib.streamkl_launch_count())
 
 
-BWD_ALGOS = {"auto": 0, "fused": 1, "split": 2}
+BWD_ALGOS = {"auto": 0, "fused": 1, "split": 2, "fused_key_tiles": 3, "fused_query_tiles": 4}
 
 
 def set_bwd_algorithm(name: str) -> None:
-    """Process-wide backward algorithm: "auto", "fused" or "split"."""
+    """Process-wide backward algorithm: "auto", "fused", "split", "fused_key_tiles" or
+    "fused_query_tiles" (see streamkl_bwd_algorithm in include/streamkl.h)."""
     st = _lib.streamkl_set_bwd_algorithm(BWD_ALGOS[name])
     if st != OK:
         raise StreamKLError(st, "streamkl_set_bwd_algorithm")

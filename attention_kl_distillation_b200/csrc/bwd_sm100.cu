@@ -696,15 +696,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
   }
 }
 
-// Per-row records for the backward, field-major per 64-row step
+// Per-row records for the key-tile backward, field-major per 64-row step
 // ([bh][step][field][64]): -LSE1*log2e, -LSE2*log2e, -L, s1*dL, s2*dL, 0, 0, 0.
 // Rows past NQ (padding of the last step) get all zeros, so their weight is
-// zero and they contribute nothing.  Also zeroes the dQ accumulator and the
-// work-unit counter that follows the records.
+// zero and they contribute nothing.  Without a record buffer (the query-tile
+// kernel) only the zeroing is done.  Also zeroes the fp32 accumulator and the
+// two work-unit counters.
 __global__ void streamkl_bwd_prep_kernel(const BwdPrepParams p) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long nrec = static_cast<long long>(p.BH) * p.NQpad;
+  const long long nrec = p.rowrec ? static_cast<long long>(p.BH) * p.NQpad : 0;
   constexpr float kLog2e = 1.4426950408889634f;
   constexpr int S = kBwdBQ;
   for (long long r = tid; r < nrec; r += stride) {
@@ -728,9 +729,8 @@ __global__ void streamkl_bwd_prep_kernel(const BwdPrepParams p) {
   for (long long e = tid; e < n4; e += stride)
     reinterpret_cast<float4*>(p.dQacc)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (tid == 0) {
-    int* counters = reinterpret_cast<int*>(p.rowrec + nrec * kRowRec);
-    counters[0] = 0;
-    counters[1] = 0;
+    p.counters[0] = 0;
+    p.counters[1] = 0;
   }
 }
 

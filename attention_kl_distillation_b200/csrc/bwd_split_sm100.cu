@@ -129,8 +129,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 //   dS1 = g1 P1 (ln2 (u1 - u2) - L),   dS2 = g2 (P2 - P1)
 // Visible streamed rows i satisfy lo <= i <= hi (MASK only).
 // Records come from shared memory per column (dK pass, COLREC) or are the
-// same for every column (dQ pass: the thread's own query row).
-template <bool MASK, bool COLREC>
+// same for every column (dQ pass: the thread's own query row).  G1/G2: which
+// of dS1, dS2 the pass contracts; only those are formed, and without dS2 the
+// student's exponential is not taken (dS1 needs the student only through u2).
+template <bool MASK, bool COLREC, bool G1, bool G2>
 __device__ __forceinline__ void form_ds(const uint32_t (&s1)[CPW], const uint32_t (&s2)[CPW],
                                         const float* rr, const float (&rec)[5], float c1,
                                         float c2, int lo, int hi, uint32_t (&w1)[CPW / 2],
@@ -143,9 +145,9 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[CPW], const uint32_
     if (COLREC) {
       nb1 = ld_shared_f4(rr + 0 * CB + q);
       nb2 = ld_shared_f4(rr + 1 * CB + q);
-      nL = ld_shared_f4(rr + 2 * CB + q);
-      g1 = ld_shared_f4(rr + 3 * CB + q);
-      g2 = ld_shared_f4(rr + 4 * CB + q);
+      nL = G1 ? ld_shared_f4(rr + 2 * CB + q) : float4{};
+      g1 = G1 ? ld_shared_f4(rr + 3 * CB + q) : float4{};
+      g2 = G2 ? ld_shared_f4(rr + 4 * CB + q) : float4{};
     } else {
       nb1 = make_float4(rec[0], rec[0], rec[0], rec[0]);
       nb2 = make_float4(rec[1], rec[1], rec[1], rec[1]);
@@ -161,15 +163,20 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[CPW], const uint32_
       const float2 B1 = e ? make_float2(nb1.z, nb1.w) : make_float2(nb1.x, nb1.y);
       const float2 B2 = e ? make_float2(nb2.z, nb2.w) : make_float2(nb2.x, nb2.y);
       const float2 NL = e ? make_float2(nL.z, nL.w) : make_float2(nL.x, nL.y);
-      const float2 G1 = e ? make_float2(g1.z, g1.w) : make_float2(g1.x, g1.y);
-      const float2 G2 = e ? make_float2(g2.z, g2.w) : make_float2(g2.x, g2.y);
+      const float2 Gs1 = e ? make_float2(g1.z, g1.w) : make_float2(g1.x, g1.y);
+      const float2 Gs2 = e ? make_float2(g2.z, g2.w) : make_float2(g2.x, g2.y);
       const float2 u1 = __ffma2_rn(S1, C1, B1);
       const float2 u2 = __ffma2_rn(S2, C2, B2);
       const float2 P1 = make_float2(ex2(u1.x), ex2(u1.y));
-      const float2 P2 = make_float2(ex2(u2.x), ex2(u2.y));
-      const float2 t = __ffma2_rn(__ffma2_rn(u2, NEG1, u1), LN2, NL);
-      float2 d1 = __fmul2_rn(__fmul2_rn(P1, t), G1);
-      float2 d2 = __fmul2_rn(__ffma2_rn(P1, NEG1, P2), G2);
+      float2 d1 = make_float2(0.f, 0.f), d2 = make_float2(0.f, 0.f);
+      if (G1) {
+        const float2 t = __ffma2_rn(__ffma2_rn(u2, NEG1, u1), LN2, NL);
+        d1 = __fmul2_rn(__fmul2_rn(P1, t), Gs1);
+      }
+      if (G2) {
+        const float2 P2 = make_float2(ex2(u2.x), ex2(u2.y));
+        d2 = __fmul2_rn(__ffma2_rn(P1, NEG1, P2), Gs2);
+      }
       if (MASK) {
         const bool vx = i >= lo && i <= hi, vy = i + 1 >= lo && i + 1 <= hi;
         d1.x = vx ? d1.x : 0.f;
@@ -177,15 +184,18 @@ __device__ __forceinline__ void form_ds(const uint32_t (&s1)[CPW], const uint32_
         d1.y = vy ? d1.y : 0.f;
         d2.y = vy ? d2.y : 0.f;
       }
-      w1[q / 2 + e] = pack_bf16(d1.x, d1.y);
-      w2[q / 2 + e] = pack_bf16(d2.x, d2.y);
+      if (G1) w1[q / 2 + e] = pack_bf16(d1.x, d1.y);
+      if (G2) w2[q / 2 + e] = pack_bf16(d2.x, d2.y);
     }
   }
 }
 
-template <BwdPass PASS, int D1, int D2>
+template <BwdPass PASS, int D1, int D2, int SEL>
 __global__ void __launch_bounds__(NTHREADS, 1)
     streamkl_bwd_split_kernel(const __grid_constant__ BwdSplitParams p) {
+  // SEL: the gradient sides this pass writes (1 teacher: out1, 2 student: out2,
+  // 3 both); a one-sided instance forms, stores and contracts that side's dS only.
+  constexpr bool G1 = (SEL & 1) != 0, G2 = (SEL & 2) != 0;
   using Lay = SplitLayout<PASS, D1, D2>;
   constexpr int NST = Lay::NST;
   constexpr bool DK = PASS == BwdPass::kDK;
@@ -387,10 +397,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // contiguous, 64-feature chunks 8 KB apart).
 #pragma unroll
           for (int kk = 0; kk < CB / 16; ++kk) {
-            if (p.out1)
+            if (G1)
               umma_bf16_ts(tmem_base + kColOut, dsa + kk * 16, sdesc_advance(c1m, kk * 2048), idO1,
                            (t > 0 || kk > 0));
-            if (p.out2)
+            if (G2)
               umma_bf16_ts(tmem_base + kColOut + D1, dsa + kk * 16 + 8, sdesc_advance(c2m, kk * 2048),
                            idO2, (t > 0 || kk > 0));
           }
@@ -466,12 +476,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint32_t w1[CPW / 2], w2[CPW / 2];
         const float* rr = DK ? rr_s(cs) + part * CPW : nullptr;
         if (masked)
-          form_ds<true, DK>(a, b, rr, rec, p.c1, p.c2, lo, hi, w1, w2);
+          form_ds<true, DK, G1, G2>(a, b, rr, rec, p.c1, p.c2, lo, hi, w1, w2);
         else
-          form_ds<false, DK>(a, b, rr, rec, p.c1, p.c2, lo, hi, w1, w2);
+          form_ds<false, DK, G1, G2>(a, b, rr, rec, p.c1, p.c2, lo, hi, w1, w2);
         // dS over this warpgroup's own S1 columns of the slot
-        tmem_st_32x32b_x8(scol, w1);
-        tmem_st_32x32b_x8(scol + CPW / 2, w2);
+        if (G1) tmem_st_32x32b_x8(scol, w1);
+        if (G2) tmem_st_32x32b_x8(scol + CPW / 2, w2);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -491,6 +501,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const size_t nrows = DK ? p.NK : p.NQ;
 #pragma unroll
       for (int tsel = 0; tsel < 2; ++tsel) {
+        if ((tsel == 0 && !G1) || (tsel == 1 && !G2)) continue;
         __nv_bfloat16* dst = tsel == 0 ? p.out1 : p.out2;
         constexpr int DW1 = D1 / NDS, DW2 = D2 / NDS;  // columns per warpgroup
         const int D = tsel == 0 ? D1 : D2;
@@ -533,22 +544,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <BwdPass PASS, int D1, int D2>
+template <BwdPass PASS, int D1, int D2, int SEL>
 cudaError_t launch_t(const BwdSplitParams& p, int grid, cudaStream_t stream) {
   constexpr int smem = SplitLayout<PASS, D1, D2>::alloc;
-  auto kern = streamkl_bwd_split_kernel<PASS, D1, D2>;
+  auto kern = streamkl_bwd_split_kernel<PASS, D1, D2, SEL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, NTHREADS, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
+template <BwdPass PASS, int SEL>
+cudaError_t launch_sel(const BwdSplitParams& p, int d1, int d2, int grid, cudaStream_t stream) {
+  if (d1 == 128 && d2 == 128) return launch_t<PASS, 128, 128, SEL>(p, grid, stream);
+  if (d1 == 128 && d2 == 64) return launch_t<PASS, 128, 64, SEL>(p, grid, stream);
+  if (d1 == 64 && d2 == 128) return launch_t<PASS, 64, 128, SEL>(p, grid, stream);
+  if (d1 == 64 && d2 == 64) return launch_t<PASS, 64, 64, SEL>(p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+// The instance is chosen by the outputs this pass writes (the page's gradient
+// configurations: one side only, or both).
 template <BwdPass PASS>
 cudaError_t launch_pass(const BwdSplitParams& p, int d1, int d2, int grid, cudaStream_t stream) {
-  if (d1 == 128 && d2 == 128) return launch_t<PASS, 128, 128>(p, grid, stream);
-  if (d1 == 128 && d2 == 64) return launch_t<PASS, 128, 64>(p, grid, stream);
-  if (d1 == 64 && d2 == 128) return launch_t<PASS, 64, 128>(p, grid, stream);
-  if (d1 == 64 && d2 == 64) return launch_t<PASS, 64, 64>(p, grid, stream);
+  const int sel = (p.out1 ? 1 : 0) | (p.out2 ? 2 : 0);
+  if (sel == 1) return launch_sel<PASS, 1>(p, d1, d2, grid, stream);
+  if (sel == 2) return launch_sel<PASS, 2>(p, d1, d2, grid, stream);
+  if (sel == 3) return launch_sel<PASS, 3>(p, d1, d2, grid, stream);
   return cudaErrorInvalidValue;
 }
 

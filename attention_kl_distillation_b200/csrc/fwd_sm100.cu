@@ -7,19 +7,23 @@
 //
 // B200 mapping (one CTA per SM, persistent):
 //   work unit   (bh, 128-row query tile)
-//   warp 0      TMA producer: 128-key tiles of K1/K2 into a ring of up to six
+//   warp 0      TMA producer: per unit the 128 query rows of Q1/Q2 into a
+//               staging buffer, per key tile K1/K2 into a ring of up to six
 //               stages (128-byte swizzle, no multicast)
 //   warp 1      TMEM owner and UMMA issuer: per key tile S1 = Q1 K1^T and
 //               S2 = Q2 K2^T (tcgen05.mma kind::f16, M = 128 rows, N = 128
 //               keys, fp32 accumulators).  Q lives in TMEM as the A operand,
-//               K in shared memory as B.  The S products rotate through three
-//               TMEM slots: S1 of the next key tile is queued behind S2 of this
-//               one while the reduction warps read this one, so the tensor
-//               pipe does not drain between key tiles.
+//               K in shared memory as B.  At the start of a unit this thread
+//               copies the staged Q rows into TMEM (tcgen05.cp) once the last
+//               products of the previous unit have read the old ones; the
+//               staging buffer is refilled for the next unit meanwhile.  The S
+//               products rotate through three TMEM slots: S1 of the next key
+//               tile is queued behind S2 of this one while the reduction warps
+//               read this one, so the tensor pipe does not drain between key
+//               tiles.
 //   warps 2..17 four reduction warpgroups, each owning 32 of the 128 keys of
 //               every key tile: thread r owns query row r (TMEM lane r).  At
-//               the start of a unit they copy the unit's rows of Q1 and Q2 from
-//               global memory into TMEM; per key tile each thread loads its
+//               each key tile each thread loads its
 //               32 + 32 logits with tcgen05.ld, frees the slots and applies the
 //               online update in registers (exp2 on the MUFU pipe, the softmax
 //               scale folded into the exponent argument, packed f32x2
@@ -55,23 +59,28 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D1, int D2>
 struct FwdLayout {
+  static constexpr int q1_bytes = BQ * D1 * 2;  // staged query rows, TMA -> tcgen05.cp
+  static constexpr int q2_bytes = BQ * D2 * 2;
   static constexpr int k1_bytes = BK * D1 * 2;
   static constexpr int k2_bytes = BK * D2 * 2;
   static constexpr int stage_bytes = k1_bytes + k2_bytes;
   static constexpr int handover_bytes = (NH - 1) * 5 * BQ * 4;
-  static constexpr int ks_fit = (232448 - 1024 - 512 - handover_bytes) / stage_bytes;
+  static constexpr int q_off = 0;
+  static constexpr int k_off = q_off + q1_bytes + q2_bytes;
+  static constexpr int ks_fit = (232448 - 1024 - 512 - handover_bytes - k_off) / stage_bytes;
   static constexpr int KSTAGES = ks_fit > 6 ? 6 : ks_fit;
-  static constexpr int k_off = 0;
   static constexpr int bar_off = k_off + KSTAGES * stage_bytes;
-  // barriers: qready, qfree, kfull[KS][2], kempty[KS][2], sfull[NSLOT], sempty[NSLOT], drain
-  static constexpr int nbar = 3 + 4 * KSTAGES + 2 * NSLOT;
+  // barriers: qsfull, qsempty, qdone, kfull[KS][2], kempty[KS][2], sfull[NSLOT],
+  // sempty[NSLOT], drain
+  static constexpr int nbar = 4 + 4 * KSTAGES + 2 * NSLOT;
   static constexpr int misc_off = bar_off + nbar * 8;
   static constexpr int part_off = misc_off + 16;  // key-part states [NH-1][5][BQ] fp32
   static constexpr int total = part_off + handover_bytes;
   static constexpr int alloc = total + 1024;  // slack to align the base to 1024 B
-  static_assert(KSTAGES >= 3, "key ring too shallow");
+  static_assert(KSTAGES >= 2, "key ring too shallow");
   static_assert(alloc <= 232448, "shared memory budget exceeded");
-  static_assert(k1_bytes % 1024 == 0 && k2_bytes % 1024 == 0,
+  static_assert(k1_bytes % 1024 == 0 && k2_bytes % 1024 == 0 && q1_bytes % 1024 == 0 &&
+                    q2_bytes % 1024 == 0,
                 "tiles must keep 1024-byte alignment for the 128B swizzle atoms");
   // TMEM columns
   __host__ __device__ static constexpr uint32_t s_col(int slot) { return slot * BK; }
@@ -221,36 +230,6 @@ __device__ __forceinline__ void tile_update(const uint32_t (&a)[KH], const uint3
   st.m2 = m2n;
 }
 
-// Copies this thread's query row of Q1 and Q2 ([BH][NQ][d] bf16) into TMEM
-// as the A operands of the S products: two features per 32-bit column, the
-// lower feature in the low half, Q2 after Q1's d1/2 columns.  The rows are
-// copied in chunks of 32 features, chunk g by warpgroup g mod NH, so the four
-// warpgroups share the work.  Rows past NQ are zero.
-template <int D1, int D2>
-__device__ __forceinline__ void stage_q_row(const FwdParams& p, int bh, int row, int part,
-                                            uint32_t taddr) {
-  const bool ok = row < p.NQ;
-  const size_t r = static_cast<size_t>(bh) * p.NQ + (ok ? row : 0);
-  const uint4* src1 = reinterpret_cast<const uint4*>(p.Q1 + r * D1);
-  const uint4* src2 = reinterpret_cast<const uint4*>(p.Q2 + r * D2);
-  constexpr int C1 = D1 / 32, C = (D1 + D2) / 32;
-#pragma unroll
-  for (int g = 0; g < C; ++g) {
-    if (g % NH != part) continue;
-    const uint4* src = g < C1 ? src1 + g * 4 : src2 + (g - C1) * 4;
-    uint32_t v[16];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint4 x = ok ? __ldg(src + k) : make_uint4(0u, 0u, 0u, 0u);
-      v[4 * k + 0] = x.x;
-      v[4 * k + 1] = x.y;
-      v[4 * k + 2] = x.z;
-      v[4 * k + 3] = x.w;
-    }
-    tmem_st_32x32b_x16(taddr + g * 16, v);  // 32 features = 16 columns
-  }
-}
-
 template <int D1, int D2>
 __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_constant__ FwdParams p) {
   using Lay = FwdLayout<D1, D2>;
@@ -259,11 +238,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off);
-  uint64_t* qready = bars + 0;    // this unit's Q rows are in TMEM
-  uint64_t* qfree = qready + 1;   // the UMMAs of the previous unit have read them
+  uint64_t* qsfull = bars + 0;     // a unit's Q rows have landed in the staging buffer
+  uint64_t* qsempty = qsfull + 1;  // they have been copied into TMEM
+  uint64_t* qdone = qsempty + 1;   // the UMMAs of the previous unit have read Q in TMEM
   // [KS][2]: the K1 and K2 halves of a stage are filled and freed separately,
   // so K1 of a later key tile is in flight as soon as S1 has read this one
-  uint64_t* kfull = qfree + 1;
+  uint64_t* kfull = qdone + 1;
   uint64_t* kempty = kfull + 2 * KS;
   uint64_t* sfull = kempty + 2 * KS;  // [NSLOT]
   uint64_t* sempty = sfull + NSLOT;   // [NSLOT]
@@ -277,8 +257,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(qready, 4 * NH);  // every reduction warp wrote its share of the Q rows
-    mbar_init(qfree, 1);
+    mbar_init(qsfull, 1);
+    mbar_init(qsempty, 1);
+    mbar_init(qdone, 1);
     for (int s = 0; s < 2 * KS; ++s) {
       mbar_init(&kfull[s], 1);
       mbar_init(&kempty[s], 1);
@@ -289,6 +270,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     }
     mbar_init(drain, 1);
     fence_mbar_init();
+    tma_prefetch_desc(&p.tmQ1);
+    tma_prefetch_desc(&p.tmQ2);
     tma_prefetch_desc(&p.tmK1);
     tma_prefetch_desc(&p.tmK2);
   }
@@ -303,6 +286,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
 
   Sched sched{fwd_units(p.BH, p.NQ, p.nsplit), static_cast<int>(gridDim.x),
               static_cast<int>(blockIdx.x), 0};
+  uint8_t* q1_s = smem + Lay::q_off;
+  uint8_t* q2_s = q1_s + Lay::q1_bytes;
   auto k1_s = [&](int s) { return smem + Lay::k_off + s * Lay::stage_bytes; };
   auto k2_s = [&](int s) { return smem + Lay::k_off + s * Lay::stage_bytes + Lay::k1_bytes; };
 
@@ -310,13 +295,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int ks = 0;
-      uint32_t kph = 0;
+      uint32_t kph = 0, qph = 0;
       uint32_t armed_k[2 * KS] = {};  // last armed phase + 1 (0 = never)
+      uint32_t armed_q = 0;
       int u;
       bool ok = true;
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
         if (w.nkt <= w.kt_lo) continue;  // split chunk past every row's frontier
+        // This unit's query rows (rows past NQ are zero-filled), once the
+        // previous unit's rows have been copied out of the staging buffer.
+        if (!(ok = mbar_wait(qsempty, qph ^ 1, ctl))) break;
+        mbar_arrive_expect_tx(qsfull, Lay::q1_bytes + Lay::q2_bytes);
+#pragma unroll
+        for (int b = 0; b < D1 / 64; ++b)
+          tma_load_3d(q1_s + b * (BQ * 128), &p.tmQ1, qsfull, b * 64, w.q0, w.bh);
+#pragma unroll
+        for (int b = 0; b < D2 / 64; ++b)
+          tma_load_3d(q2_s + b * (BQ * 128), &p.tmQ2, qsfull, b * 64, w.q0, w.bh);
+        armed_q = qph + 1;
+        qph ^= 1;
         for (int kt = w.kt_lo; kt < (p.withhold_keys ? w.kt_lo : w.nkt); ++kt) {
           if (!(ok = mbar_wait(&kempty[2 * ks], kph ^ 1, ctl))) break;
           mbar_arrive_expect_tx(&kfull[2 * ks], Lay::k1_bytes);
@@ -342,6 +340,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
         WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
         for (int s = 0; s < 2 * KS; ++s)
           if (armed_k[s]) mbar_wait(&kfull[s], armed_k[s] - 1, dctl);
+        if (armed_q) mbar_wait(qsfull, armed_q - 1, dctl);
       }
     }
   } else if (warp == 1) {
@@ -349,17 +348,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(BQ, BK);
       const uint32_t a1 = tmem_base + Lay::q_col, a2 = a1 + D1 / 2;
+      const uint64_t q1sd = sdesc_sw128(smem_u32(q1_s), 16, 1024);
+      const uint64_t q2sd = sdesc_sw128(smem_u32(q2_s), 16, 1024);
       int ks = 0;
-      uint32_t kph = 0, qph = 0;
+      uint32_t kph = 0, qsph = 0, qdph = 0;
+      bool first = true;
       SlotRing ring;
       int u;
       bool ok = true;
       while (ok && sched.next(u)) {
         const Unit w = decode_unit(p, u);
         if (w.nkt <= w.kt_lo) continue;
-        if (!(ok = mbar_wait(qready, qph, ctl))) break;  // Q of this unit is in TMEM
-        qph ^= 1;
+        if (!first) {
+          // The previous unit's products must have read Q out of TMEM before
+          // it is overwritten (a copy is not ordered after earlier products).
+          umma_commit(qdone);
+          if (!(ok = mbar_wait(qdone, qdph, ctl))) break;
+          qdph ^= 1;
+        }
+        first = false;
+        if (!(ok = mbar_wait(qsfull, qsph, ctl))) break;  // Q rows of this unit staged
+        qsph ^= 1;
         tc_fence_after();
+        // Staged rows into TMEM, one 16-feature slice per copy at the columns the
+        // products read it from; the products issued below see the copies.
+#pragma unroll
+        for (int kk = 0; kk < D1 / 16; ++kk)
+          tmem_cp_128x256b(a1 + kk * 8, sdesc_advance(q1sd, (kk >> 2) * (BQ * 128) + (kk & 3) * 32));
+#pragma unroll
+        for (int kk = 0; kk < D2 / 16; ++kk)
+          tmem_cp_128x256b(a2 + kk * 8, sdesc_advance(q2sd, (kk >> 2) * (BQ * 128) + (kk & 3) * 32));
+        umma_commit(qsempty);  // the staging buffer is free once the copies are done
         for (int kt = w.kt_lo; kt < w.nkt; ++kt) {
           // Descriptors built once per stage; each UMMA below costs an add and the
           // MMA itself, so this thread keeps up although it shares its SM
@@ -400,7 +419,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
           }
         }
         if (!ok) break;
-        umma_commit(qfree);  // once this unit's UMMAs are done
       }
       // Every UMMA issued by this thread completes before TMEM is released.
       umma_commit(drain);
@@ -416,7 +434,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
     const uint32_t tlane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     float* part = reinterpret_cast<float*>(smem + Lay::part_off);
     const int off = p.NK - p.NQ;
-    uint32_t qfph = 0;
     SlotRing ring;
     int u;
     bool ok = true;
@@ -424,15 +441,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_fwd_kernel(const __grid_
       const Unit w = decode_unit(p, u);
       if (w.nkt <= w.kt_lo) continue;
       const int i_abs = w.q0 + row;
-      // This unit's Q rows into TMEM, once the previous unit's UMMAs have read them.
-      if (!(ok = mbar_wait(qfree, qfph ^ 1, ctl))) break;
-      qfph ^= 1;
-      tc_fence_after();
-      stage_q_row<D1, D2>(p, w.bh, i_abs, hf, tlane + Lay::q_col);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(qready);
       const int lim = p.causal ? min(p.NK, i_abs + off + 1) : p.NK;  // visible keys [0, lim)
       RowState st{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
       for (int kt = w.kt_lo; kt < w.nkt; ++kt) {

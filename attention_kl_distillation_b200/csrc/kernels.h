@@ -17,8 +17,9 @@ constexpr int kFwdBK = 128;
 
 struct FwdParams {
   CUtensorMap tmK1, tmK2;  // 3-D maps over [BH][NK][d], 128-row boxes, 128B swizzle
-  CUtensorMap tmQ1, tmQ2;  // transposed kernel only: [BH][NQ][d], boxes of one query group
-  const __nv_bfloat16* Q1;  // [BH][NQ][d1], read row by row into TMEM
+  CUtensorMap tmQ1, tmQ2;  // [BH][NQ][d], boxes of one query group (transposed kernel)
+                           // or of 128 rows (row-tile kernel)
+  const __nv_bfloat16* Q1;  // [BH][NQ][d1]
   const __nv_bfloat16* Q2;  // [BH][NQ][d2]
   float* L;
   float* LSE1;
@@ -90,20 +91,52 @@ struct BwdPrepParams {
   const float* LSE1;
   const float* LSE2;
   const float* dL;
-  float* rowrec;
-  float* dQacc;
+  float* rowrec;        // null: no per-query records (the query-tile kernel reads L/LSE itself)
+  float* dQacc;         // the fp32 accumulator to zero (dQ or dK, whichever the kernel reduces)
   long long dqacc_elems;
+  int* counters;        // two work-unit counters, zeroed
   int BH, NQ, NQpad;
   float s1, s2;
 };
 
 struct BwdConvertParams {
-  const float* dQacc;
-  __nv_bfloat16* dQ1;  // may be null
-  __nv_bfloat16* dQ2;  // may be null
-  long long rows;      // BH * NQ
+  const float* dQacc;  // fp32 [rows][d1 + d2]
+  __nv_bfloat16* dQ1;  // [rows][d1], may be null
+  __nv_bfloat16* dQ2;  // [rows][d2], may be null
+  long long rows;      // BH * NQ (dQ) or BH * NK (dK)
   int d1, d2;
 };
+
+// Query-tile variant of the fused backward: a work unit is one 128-query tile
+// (the UMMA M of S and dQ), which visits its visible keys in 64-key steps; dQ
+// stays in TMEM for the unit, dK goes through fp32 reductions into dKacc.
+constexpr int kBwdQtRows = 128;
+constexpr int kBwdQtKeys = 64;
+
+struct BwdQtParams {
+  CUtensorMap tmQ1, tmK1, tmQ2, tmK2;  // Q maps: 128-row boxes; K maps: 64-row boxes
+  const float* L;       // saved state and upstream gradient, fp32 [BH][NQ]
+  const float* LSE1;
+  const float* LSE2;
+  const float* dL;
+  float* dKacc;         // [BH][NK][ld] fp32, ld = widths of the selected sides, zeroed first
+  int* counter;         // work-unit counter, zeroed first
+  __nv_bfloat16* dQ1;   // [BH][NQ][d1] or null
+  __nv_bfloat16* dQ2;   // [BH][NQ][d2] or null
+  int BH, NQ, NK, causal;
+  int want_dq1, want_dk1, want_dq2, want_dk2;
+  float c1, c2;  // s_t * log2(e)
+  float s1, s2;
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+// sel as for launch_bwd.
+cudaError_t launch_bwd_qt(const BwdQtParams& p, int d1, int d2, int sel, int grid,
+                          cudaStream_t stream);
+__host__ __device__ inline int bwd_qt_units(int BH, int NQ) {
+  return BH * ((NQ + kBwdQtRows - 1) / kBwdQtRows);
+}
 
 // Split backward (two passes of one kernel template): the dK pass streams
 // query tiles past resident 128-key tiles, the dQ pass streams key tiles past

@@ -180,6 +180,14 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+// Copies a 128-row x 32-byte slice of a shared-memory matrix, described as for
+// a UMMA operand, into 128 TMEM lanes x 8 columns (lane r gets row r, bytes in
+// order: column j holds elements 2j and 2j+1, the lower in the low half).
+// A following tcgen05.mma issued by this thread sees the copied data.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {

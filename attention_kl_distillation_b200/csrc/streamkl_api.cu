@@ -166,9 +166,10 @@ float scale_or_default(float s, int d) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Backward workspace: fp32 dQ accumulator [BH][NQ][d1+d2], then the per-row
-// records [BH][NQpad][8] fp32, then the work-unit counter; each part starts on
-// a 256-byte boundary.
+// Backward workspace: the fp32 accumulator of the reduced gradient ([BH][NQ][ld]
+// dQ for key-tile units, [BH][NK][ld] dK for query-tile units; sized for the
+// larger), then the per-row records [BH][NQpad][8] fp32, then two work-unit
+// counters; each part starts on a 256-byte boundary.
 struct BwdWorkspace {
   size_t dqacc_elems, rowrec_off, counter_off, total;
   int NQpad;
@@ -184,6 +185,8 @@ int bwd_algo_setting() {
     if (const char* e = std::getenv("STREAMKL_BWD_ALGO")) {
       if (!std::strcmp(e, "fused")) a = STREAMKL_BWD_FUSED;
       else if (!std::strcmp(e, "split")) a = STREAMKL_BWD_SPLIT;
+      else if (!std::strcmp(e, "fused_key_tiles")) a = STREAMKL_BWD_FUSED_KEY_TILES;
+      else if (!std::strcmp(e, "fused_query_tiles")) a = STREAMKL_BWD_FUSED_QUERY_TILES;
     }
     int expect = -1;
     // a concurrent streamkl_set_bwd_algorithm wins over the environment default
@@ -200,12 +203,37 @@ int bwd_algo_setting() {
 // above every measured shape; set the algorithm explicitly to override.
 constexpr size_t kFusedDqAccLimit = 4ull << 30;
 
+// SMs of the current device for scheduling decisions; 148 (B200) when no
+// device can be queried, so that the decision is the same on a host without one.
+int sms_or_default() {
+  int dev = -1, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+    return n;
+  cudaGetLastError();
+  return 148;
+}
+
+// Fused orientation: query-tile units (dQ on chip, dK reduced) when there are
+// enough of them to fill the SMs twice over, else key-tile units (dK on chip,
+// dQ reduced), which have more units when N_Q is small.
+streamkl_bwd_algorithm fused_orientation(const streamkl_problem& pr) {
+  const int64_t BH = static_cast<int64_t>(pr.B) * pr.H;
+  const int64_t units_q = BH * ((pr.NQ + skl::kBwdQtRows - 1) / skl::kBwdQtRows);
+  return units_q >= 2 * static_cast<int64_t>(sms_or_default()) ? STREAMKL_BWD_FUSED_QUERY_TILES
+                                                               : STREAMKL_BWD_FUSED_KEY_TILES;
+}
+
+// The concrete algorithm: SPLIT, FUSED_KEY_TILES or FUSED_QUERY_TILES.
 streamkl_bwd_algorithm resolve_bwd_algo(const streamkl_problem& pr) {
   const int a = bwd_algo_setting();
-  if (a == STREAMKL_BWD_FUSED || a == STREAMKL_BWD_SPLIT) return static_cast<streamkl_bwd_algorithm>(a);
+  if (a == STREAMKL_BWD_SPLIT || a == STREAMKL_BWD_FUSED_KEY_TILES ||
+      a == STREAMKL_BWD_FUSED_QUERY_TILES)
+    return static_cast<streamkl_bwd_algorithm>(a);
+  if (a == STREAMKL_BWD_FUSED) return fused_orientation(pr);
   const size_t acc = static_cast<size_t>(pr.B) * pr.H * static_cast<size_t>(pr.NQ) *
                      static_cast<size_t>(pr.d1 + pr.d2) * sizeof(float);
-  return acc > kFusedDqAccLimit ? STREAMKL_BWD_SPLIT : STREAMKL_BWD_FUSED;
+  return acc > kFusedDqAccLimit ? STREAMKL_BWD_SPLIT : fused_orientation(pr);
 }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -214,7 +242,8 @@ BwdWorkspace bwd_workspace_layout(const streamkl_problem& pr) {
   BwdWorkspace w;
   const size_t BH = static_cast<size_t>(pr.B) * pr.H;
   w.NQpad = (pr.NQ + skl::kBwdBQ - 1) / skl::kBwdBQ * skl::kBwdBQ;
-  w.dqacc_elems = BH * static_cast<size_t>(pr.NQ) * static_cast<size_t>(pr.d1 + pr.d2);
+  w.dqacc_elems = BH * static_cast<size_t>(pr.NQ > pr.NK ? pr.NQ : pr.NK) *
+                  static_cast<size_t>(pr.d1 + pr.d2);
   w.rowrec_off = round256(w.dqacc_elems * sizeof(float));
   const size_t rec = BH * static_cast<size_t>(w.NQpad) * skl::kRowRec * sizeof(float);
   w.counter_off = w.rowrec_off + rec;  // two work-unit counters follow the records
@@ -249,7 +278,8 @@ streamkl_status streamkl_debug_inject(int mode) {
 }
 
 streamkl_status streamkl_set_bwd_algorithm(streamkl_bwd_algorithm algo) {
-  if (algo != STREAMKL_BWD_AUTO && algo != STREAMKL_BWD_FUSED && algo != STREAMKL_BWD_SPLIT)
+  if (algo != STREAMKL_BWD_AUTO && algo != STREAMKL_BWD_FUSED && algo != STREAMKL_BWD_SPLIT &&
+      algo != STREAMKL_BWD_FUSED_KEY_TILES && algo != STREAMKL_BWD_FUSED_QUERY_TILES)
     return STREAMKL_EINVAL;
   g_bwd_algo.store(algo);
   return STREAMKL_OK;
@@ -307,11 +337,11 @@ streamkl_status prepare_fwd(const streamkl_problem* prob, const void* Q1, const 
   const int64_t BH = static_cast<int64_t>(prob->B) * prob->H;
   if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kFwdBK, &p->tmK1)) != STREAMKL_OK) return st;
   if ((st = tensor_map(K2, BH, prob->NK, prob->d2, skl::kFwdBK, &p->tmK2)) != STREAMKL_OK) return st;
-  if (prob->NQ <= skl::kFwdTMaxNQ) {  // transposed kernel: Q groups are TMA boxes
-    const int nqt = skl::fwd_t_rows(prob->NQ);
-    if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, nqt, &p->tmQ1)) != STREAMKL_OK) return st;
-    if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, nqt, &p->tmQ2)) != STREAMKL_OK) return st;
-  }
+  // Q tiles are TMA boxes: a query group of the transposed kernel, or the 128
+  // rows of a row-tile unit (staged in shared memory, then copied into TMEM).
+  const int qrows = prob->NQ <= skl::kFwdTMaxNQ ? skl::fwd_t_rows(prob->NQ) : skl::kFwdBQ;
+  if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, qrows, &p->tmQ1)) != STREAMKL_OK) return st;
+  if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, qrows, &p->tmQ2)) != STREAMKL_OK) return st;
   p->Q1 = static_cast<const __nv_bfloat16*>(Q1);
   p->Q2 = static_cast<const __nv_bfloat16*>(Q2);
   p->L = L;
@@ -525,21 +555,26 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   float* rowrec = reinterpret_cast<float*>(ws + lay.rowrec_off);
   const float s1 = scale_or_default(prob->s1, prob->d1);
   const float s2 = scale_or_default(prob->s2, prob->d2);
-  const bool split = resolve_bwd_algo(*prob) == STREAMKL_BWD_SPLIT;
-  const bool want_dq = (dQ1 || dQ2) && !split;  // the fused path accumulates dQ in fp32
-  // Gradient sides asked for (the page's configurations): the fused kernel is
-  // specialised on them and its dQ accumulator holds only their columns.
+  const streamkl_bwd_algorithm algo = resolve_bwd_algo(*prob);
+  const bool split = algo == STREAMKL_BWD_SPLIT;
+  const bool qtiles = algo == STREAMKL_BWD_FUSED_QUERY_TILES;
+  // the fused kernels accumulate one gradient in fp32: dQ over key tiles, dK over query tiles
+  const bool want_acc = !split && (qtiles ? (dK1 || dK2) : (dQ1 || dQ2));
+  // Gradient sides asked for (the page's configurations): the fused kernels are
+  // specialised on them and their accumulator holds only those sides' columns.
   const int sel = ((dQ1 || dK1) ? 1 : 0) | ((dQ2 || dK2) ? 2 : 0);
   const int ld1 = (sel & 1) ? prob->d1 : 0, ld2 = (sel & 2) ? prob->d2 : 0;
+  int* counters = reinterpret_cast<int*>(ws + lay.counter_off);
 
   skl::BwdPrepParams pp;
   pp.L = L;
   pp.LSE1 = LSE1;
   pp.LSE2 = LSE2;
   pp.dL = dL;
-  pp.rowrec = rowrec;
+  pp.rowrec = qtiles ? nullptr : rowrec;  // the query-tile kernel reads L, LSE and dL itself
   pp.dQacc = dqacc;
-  pp.dqacc_elems = want_dq ? BH * static_cast<int64_t>(prob->NQ) * (ld1 + ld2) : 0;
+  pp.dqacc_elems = want_acc ? BH * static_cast<int64_t>(qtiles ? prob->NK : prob->NQ) * (ld1 + ld2) : 0;
+  pp.counters = counters;
   pp.BH = static_cast<int>(BH);
   pp.NQ = prob->NQ;
   pp.NQpad = lay.NQpad;
@@ -549,7 +584,6 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   g_launches.fetch_add(1);
 
   if (split) {
-    int* counters = reinterpret_cast<int*>(ws + lay.counter_off);
     skl::BwdSplitParams sp;
     sp.rowrec = rowrec;
     sp.BH = static_cast<int>(BH);
@@ -592,6 +626,52 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
     return STREAMKL_OK;
   }
 
+  if (qtiles) {
+    skl::BwdQtParams p;
+    if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, skl::kBwdQtRows, &p.tmQ1)) != STREAMKL_OK) return st;
+    if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kBwdQtKeys, &p.tmK1)) != STREAMKL_OK) return st;
+    if ((st = tensor_map(Q2, BH, prob->NQ, prob->d2, skl::kBwdQtRows, &p.tmQ2)) != STREAMKL_OK) return st;
+    if ((st = tensor_map(K2, BH, prob->NK, prob->d2, skl::kBwdQtKeys, &p.tmK2)) != STREAMKL_OK) return st;
+    p.L = L;
+    p.LSE1 = LSE1;
+    p.LSE2 = LSE2;
+    p.dL = dL;
+    p.dKacc = dqacc;
+    p.counter = counters;
+    p.dQ1 = static_cast<__nv_bfloat16*>(dQ1);
+    p.dQ2 = static_cast<__nv_bfloat16*>(dQ2);
+    p.BH = static_cast<int>(BH);
+    p.NQ = prob->NQ;
+    p.NK = prob->NK;
+    p.causal = prob->causal;
+    p.want_dq1 = dQ1 != nullptr;
+    p.want_dk1 = dK1 != nullptr;
+    p.want_dq2 = dQ2 != nullptr;
+    p.want_dk2 = dK2 != nullptr;
+    p.c1 = s1 * kLog2e;
+    p.c2 = s2 * kLog2e;
+    p.s1 = s1;
+    p.s2 = s2;
+    p.status = dev->status;
+    p.wait_limit_ns = wait_limit_ns();
+    const int units = skl::bwd_qt_units(p.BH, p.NQ);
+    const int grid = units < dev->num_sms ? units : dev->num_sms;
+    if (skl::launch_bwd_qt(p, prob->d1, prob->d2, sel, grid, s) != cudaSuccess) return STREAMKL_ECUDA;
+    g_launches.fetch_add(1);
+    if (want_acc) {
+      skl::BwdConvertParams cp;
+      cp.dQacc = dqacc;
+      cp.dQ1 = static_cast<__nv_bfloat16*>(dK1);
+      cp.dQ2 = static_cast<__nv_bfloat16*>(dK2);
+      cp.rows = BH * prob->NK;
+      cp.d1 = ld1;  // accumulator columns: teacher side (if selected), then student side
+      cp.d2 = ld2;
+      if (skl::launch_bwd_convert(cp, dev->num_sms, s) != cudaSuccess) return STREAMKL_ECUDA;
+      g_launches.fetch_add(1);
+    }
+    return STREAMKL_OK;
+  }
+
   skl::BwdParams p;
   if ((st = tensor_map(Q1, BH, prob->NQ, prob->d1, skl::kBwdBQ, &p.tmQ1)) != STREAMKL_OK) return st;
   if ((st = tensor_map(K1, BH, prob->NK, prob->d1, skl::kBwdBK, &p.tmK1)) != STREAMKL_OK) return st;
@@ -619,7 +699,7 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   if (skl::launch_bwd(p, prob->d1, prob->d2, sel, grid, s) != cudaSuccess) return STREAMKL_ECUDA;
   g_launches.fetch_add(1);
 
-  if (want_dq) {
+  if (want_acc) {
     skl::BwdConvertParams cp;
     cp.dQacc = dqacc;
     cp.dQ1 = static_cast<__nv_bfloat16*>(dQ1);

@@ -67,6 +67,9 @@ def parse_args(argv=None):
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N > 1: every rank runs the whole workload (replicas, weak scaling) or "
                          "a contiguous range of its B*H heads (heads, strong scaling)")
+    ap.add_argument("--bwd-algo", default="auto",
+                    choices=["auto", "fused", "split", "fused_key_tiles", "fused_query_tiles"],
+                    help="streamkl_bwd algorithm (process-wide setting of the library)")
     ap.add_argument("--need", default="1111",
                     help="which of dQ1 dK1 dQ2 dK2 the backward returns (e.g. 0101 = dK only)")
     return ap.parse_args(argv)
@@ -117,7 +120,8 @@ def run_config(args, w: Workload, phase: str, world: int, nsplit=None) -> dict:
 PROFILED_SOURCES = {
     "fwd_kernel": "fwd_sm100.cu",
     "fwd_t_kernel": "fwd_t_sm100.cu",
-    "bwd_fused_kernel": "bwd_sm100.cu",
+    "bwd_fused_key_tiles_kernel": "bwd_sm100.cu",
+    "bwd_fused_query_tiles_kernel": "bwd_qt_sm100.cu",
     "bwd_split_kernel": "bwd_split_sm100.cu",
 }
 
@@ -322,28 +326,32 @@ def run_table(args):
         grads = tuple(torch.empty_like(t) for t in (Q1, K1, Q2, K2)) if w.backward else None
         ws = (torch.empty(binding.workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal),
                           dtype=torch.uint8, device=dev) if w.backward else None)
-        calls = [("fwd", lambda: skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B)), w.fwd_flops())]
+        calls = [("fwd", None, lambda: skl.fwd(Q1, K1, Q2, K2, causal=w.causal, out=(L, A, B)),
+                  w.fwd_flops())]
         ns = binding.splitk_suggest(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal)
         if ns > 1 and name != "tiny":
             fws = torch.empty(max(256, binding.splitk_workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, ns)),
                               dtype=torch.uint8, device=dev)
-            calls.append((f"fwd_splitk{ns}",
+            calls.append((f"fwd_splitk{ns}", None,
                           lambda: skl.fwd_splitk(Q1, K1, Q2, K2, causal=w.causal, nsplit=ns,
                                                  workspace=fws, out=(L, A, B)), w.fwd_flops()))
         if w.backward:
-            calls.append(("bwd", lambda: skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal,
-                                                 workspace=ws, out=grads), w.bwd_flops()))
+            for algo in ("fused_key_tiles", "fused_query_tiles", "split"):
+                calls.append((f"bwd_{algo}", algo,
+                              lambda: skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal,
+                                              workspace=ws, out=grads), w.bwd_flops()))
             # one gradient side (teacher fixed: dQ2, dK2; student fixed: dQ1, dK1): both S
             # products are recomputed, the contractions of the other side are not done
             pairs = w.bwd_flops() / (6 * (w.d1 + w.d2))
             for side, keep, d in (("student", (2, 3), w.d2), ("teacher", (0, 1), w.d1)):
                 outs = tuple(g if i in keep else None for i, g in enumerate(grads))
-                calls.append((f"bwd_{side}_side",
+                calls.append((f"bwd_{side}_side", None,
                               lambda outs=outs: skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal,
                                                         workspace=ws, out=outs),
                               pairs * (2 * (w.d1 + w.d2) + 4 * d)))
         n = 5 if name == "long64k" else 10
-        for phase, fn, fl in calls:
+        for phase, algo, fn, fl in calls:
+            binding.set_bwd_algorithm(algo or args.bwd_algo)
             for _ in range(3):
                 fn()
             times = []
@@ -395,6 +403,7 @@ def main(argv=None):
     import attention_kl_distillation_b200 as skl
     from attention_kl_distillation_b200 import binding
     from attention_kl_distillation_b200.parallel import max_over_ranks
+    binding.set_bwd_algorithm(args.bwd_algo)
 
     dev = torch.device("cuda", local)
     full_w = w

@@ -113,10 +113,11 @@ size_t streamkl_fwd_splitk_workspace_size(const streamkl_problem *prob, int nspl
 int streamkl_fwd_splitk_suggest(const streamkl_problem *prob);
 
 /*
- * Workspace bytes that streamkl_bwd needs for this problem: an fp32 dQ
- * accumulator [B][H][NQ][d1+d2] (section 2, "Fusione del Kernel": dQ is
- * accumulated with atomics across key tiles) plus padding.  0 on a bad
- * problem.
+ * Workspace bytes that streamkl_bwd needs for this problem: an fp32
+ * accumulator for the gradient the fused kernels reduce across tiles (section
+ * 2, "Fusione del Kernel": dQ with atomics across key tiles, or dK across
+ * query tiles), [B][H][max(NQ,NK)][d1+d2], plus per-row records and padding.
+ * The same size serves every algorithm.  0 on a bad problem.
  */
 size_t streamkl_bwd_workspace_size(const streamkl_problem *prob);
 
@@ -186,28 +187,39 @@ streamkl_status streamkl_bwd_noalloc(const streamkl_problem *prob, const float *
 /*
  * How streamkl_bwd computes the gradients (section 2, "Fusione del Kernel",
  * and the fused-versus-separate ablation):
- *  FUSED  one kernel visits every (query tile, key tile) pair once; dK stays
- *         on chip, dQ is accumulated across key tiles with fp32 reductions
- *         into the workspace, then converted to bf16.
- *  SPLIT  two passes of one kernel: a dK pass over key tiles and a dQ pass
- *         over query tiles, each regenerating the probabilities; no
- *         reductions in global memory.
- *  AUTO   FUSED unless the fp32 dQ accumulator (B*H*NQ*(d1+d2)*4 bytes)
- *         exceeds 4 GiB; on B200 the fused kernel measured faster at every
- *         size tested.
+ *  FUSED_KEY_TILES    one kernel visits every (query tile, key tile) pair
+ *                     once, with 128-key work units; dK stays on chip, dQ is
+ *                     accumulated across key tiles with fp32 reductions into
+ *                     the workspace (the page's design), then converted.
+ *  FUSED_QUERY_TILES  the same with 128-query work units: dQ stays on chip and
+ *                     dK is accumulated across query tiles with fp32
+ *                     reductions.  Each dS thread then owns a query row, so
+ *                     its L, LSE and dL are registers instead of shared-memory
+ *                     loads for every key.
+ *  FUSED              the fused orientation chosen by shape: query tiles when
+ *                     B*H*ceil(NQ/128) fills the device's SMs twice, else key
+ *                     tiles.
+ *  SPLIT              two passes of one kernel: a dK pass over key tiles and
+ *                     a dQ pass over query tiles, each regenerating the
+ *                     probabilities; no reductions in global memory.
+ *  AUTO               FUSED unless the fp32 accumulator (B*H*NQ*(d1+d2)*4
+ *                     bytes) exceeds 4 GiB, then SPLIT.
  * Results agree within rounding either way.  Process-wide; default AUTO (or
- * the environment variable STREAMKL_BWD_ALGO = auto | fused | split, read
- * once).
+ * the environment variable STREAMKL_BWD_ALGO = auto | fused | split |
+ * fused_key_tiles | fused_query_tiles, read once).
  */
 typedef enum {
   STREAMKL_BWD_AUTO = 0,
   STREAMKL_BWD_FUSED = 1,
-  STREAMKL_BWD_SPLIT = 2
+  STREAMKL_BWD_SPLIT = 2,
+  STREAMKL_BWD_FUSED_KEY_TILES = 3,
+  STREAMKL_BWD_FUSED_QUERY_TILES = 4
 } streamkl_bwd_algorithm;
 
 streamkl_status streamkl_set_bwd_algorithm(streamkl_bwd_algorithm algo);
 
-/* The algorithm streamkl_bwd would use for this problem (AUTO resolved). */
+/* The algorithm streamkl_bwd would use for this problem on the current device:
+ * SPLIT, FUSED_KEY_TILES or FUSED_QUERY_TILES (AUTO and FUSED resolved). */
 streamkl_bwd_algorithm streamkl_bwd_algorithm_for(const streamkl_problem *prob);
 
 /* Static English text for a status code. */

@@ -61,7 +61,7 @@ def test_fwd_rejects_nonfinite_scale():
 
 def test_workspace_size():
     ws = B.workspace_size(2, 3, 100, 50, 128, 64)
-    need = 2 * 3 * 100 * (128 + 64) * 4 + 2 * 3 * 128 * 8 * 4   # dQ accumulator + row records
+    need = 2 * 3 * 100 * (128 + 64) * 4 + 2 * 3 * 128 * 8 * 4   # accumulator + row records
     assert ws >= need and ws % 256 == 0 and ws - need <= 768
     assert B.workspace_size(1, 1, 0, 5, 64, 64) == 0
     assert B.workspace_size(1, 1, 5, 5, 96, 64) == 0
@@ -109,17 +109,24 @@ def test_binding_argtypes_match_header():
 
 
 def test_bwd_algorithm_selection():
+    """bwd_algorithm_for resolves AUTO and FUSED to a concrete algorithm.  Without a GPU
+    the device is taken to have 148 SMs, as a B200 does."""
     lib = B.lib()
     assert lib.streamkl_set_bwd_algorithm(7) == B.EINVAL
     try:
+        for name in ("split", "fused_key_tiles", "fused_query_tiles"):
+            B.set_bwd_algorithm(name)
+            assert B.bwd_algorithm_for(1, 2, 256, 256, 64, 64) == name
         B.set_bwd_algorithm("fused")
-        assert B.bwd_algorithm_for(1, 32, 16384, 16384, 128, 128, True) == "fused"
-        B.set_bwd_algorithm("split")
-        assert B.bwd_algorithm_for(1, 2, 256, 256, 64, 64) == "split"
+        # query tiles once B*H*ceil(NQ/128) fills the SMs twice (296 units), else key tiles
+        assert B.bwd_algorithm_for(1, 32, 16384, 16384, 128, 128, True) == "fused_query_tiles"
+        assert B.bwd_algorithm_for(1, 32, 1024, 32768, 128, 128, True) == "fused_key_tiles"
+        assert B.bwd_algorithm_for(1, 37, 1024, 1024, 128, 128) == "fused_query_tiles"
+        assert B.bwd_algorithm_for(1, 36, 1024, 1024, 128, 128) == "fused_key_tiles"
         B.set_bwd_algorithm("auto")
-        # AUTO: fused unless the fp32 dQ accumulator exceeds 4 GiB
-        assert B.bwd_algorithm_for(1, 2, 256, 256, 64, 64) == "fused"
-        assert B.bwd_algorithm_for(1, 32, 16384, 16384, 128, 128, True) == "fused"
+        # AUTO: fused unless the fp32 accumulator exceeds 4 GiB
+        assert B.bwd_algorithm_for(1, 2, 256, 256, 64, 64) == "fused_key_tiles"
+        assert B.bwd_algorithm_for(1, 32, 16384, 16384, 128, 128, True) == "fused_query_tiles"
         assert B.bwd_algorithm_for(4, 32, 65536, 65536, 128, 128, True) == "split"
     finally:
         B.set_bwd_algorithm("auto")

@@ -66,15 +66,15 @@ def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", tmp_path)
     sha = bench.kernel_sources_sha1("bwd_sm100.cu")
-    prof = tmp_path / "profiles" / "bwd_fused_kernel_case.md"
+    prof = tmp_path / "profiles" / "bwd_fused_key_tiles_kernel_case.md"
     prof.write_text(f"source-sha1: {sha}\n- dram-bytes-per-full-launch: 12345\n")
-    assert bench.profiled_traffic("bwd_fused_kernel_case.md") == 12345
+    assert bench.profiled_traffic("bwd_fused_key_tiles_kernel_case.md") == 12345
     # another kernel's file does not matter
     (csrc / "fwd_sm100.cu").write_text("// changed\n")
-    assert bench.profiled_traffic("bwd_fused_kernel_case.md") == 12345
+    assert bench.profiled_traffic("bwd_fused_key_tiles_kernel_case.md") == 12345
     # the profiled kernel's own file or a shared header does
     (csrc / "sm100.cuh").write_text("// changed\n")
-    assert bench.profiled_traffic("bwd_fused_kernel_case.md") is None
+    assert bench.profiled_traffic("bwd_fused_key_tiles_kernel_case.md") is None
     assert bench.profiled_traffic("missing.md") is None
 
 

@@ -8,9 +8,10 @@ from gpu_common import TOL_GRAD, check_fwd, cuda_inputs, oracle_bits, rel_froben
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["fused", "split"])
+@pytest.fixture(autouse=True, params=["fused_key_tiles", "fused_query_tiles", "split"])
 def bwd_algo(request):
-    """Every backward test runs with both algorithms of streamkl_bwd."""
+    """Every backward test runs with each algorithm of streamkl_bwd: the fused kernel
+    with key-tile units and with query-tile units, and the two split passes."""
     from attention_kl_distillation_b200 import set_bwd_algorithm
     set_bwd_algorithm(request.param)
     yield request.param
@@ -41,6 +42,24 @@ def run_bwd(dev, dL, causal, need=(True, True, True, True), s1=None, s2=None, sa
         BH = L.shape[0] * L.shape[1]
         return out, tuple(t.reshape(BH, -1).cpu().numpy().astype(np.float64) for t in (L, A, B))
     return out
+
+
+_FWDBWD_ORACLE = {}
+
+
+def fwdbwd16k_oracle(orc, bits, kind, key, g):
+    """Oracle results on the forward+backward workload, computed once per session:
+    every backward algorithm is checked against the same rows and heads."""
+    if (kind, key) not in _FWDBWD_ORACLE:
+        if kind == "rows":
+            rows = np.asarray(key, dtype=np.int64).reshape(-1, 2)
+            _FWDBWD_ORACLE[(kind, key)] = orc.bwd_rows(*bits, rows, np.full(len(rows), g),
+                                                       causal=True)
+        else:
+            _FWDBWD_ORACLE[(kind, key)] = orc.bwd_heads(*bits, list(key),
+                                                        np.full((len(key), bits[0].shape[2]), g),
+                                                        causal=True)
+    return _FWDBWD_ORACLE[(kind, key)]
 
 
 def oracle_heads(orc, ins, dL, causal, heads, s1=None, s2=None):
@@ -115,21 +134,24 @@ def test_bwd_one_sided_and_partial_outputs(orc, need, dims):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-def test_bwd_one_sided_dk_matches_full_kernel_bitwise(bwd_algo, causal):
-    """dK is accumulated in TMEM in a fixed order, and a one-sided kernel forms
-    its dS with the same arithmetic as the two-sided one, so its dK is the
-    same to the bit (dQ goes through fp32 atomics and is not compared)."""
-    if bwd_algo != "fused":
+def test_bwd_one_sided_matches_full_kernel_bitwise(bwd_algo, causal):
+    """The gradient a fused kernel keeps on chip (dK with key-tile units, dQ with
+    query-tile units) is accumulated in TMEM in a fixed order, and a one-sided
+    kernel forms its dS with the same arithmetic as the two-sided one, so that
+    gradient is the same to the bit (the other goes through fp32 atomics and is
+    not compared)."""
+    if not bwd_algo.startswith("fused"):
         pytest.skip("the specialised kernels are the fused path")
     from attention_kl_distillation_b200.inputs import make_inputs
     w = workload(1, 2, 192, 320, 128, 128, causal)
     dev = cuda_inputs(make_inputs(w))
     dL = torch.randn((1, 2, w.NQ), device="cuda")
     full = run_bwd(dev, dL, causal)
-    teacher = run_bwd(dev, dL, causal, need=(False, True, False, False))
-    student = run_bwd(dev, dL, causal, need=(False, False, False, True))
-    assert np.array_equal(teacher[1], full[1])
-    assert np.array_equal(student[3], full[3])
+    i1, i2 = (1, 3) if bwd_algo == "fused_key_tiles" else (0, 2)
+    teacher = run_bwd(dev, dL, causal, need=tuple(k == i1 for k in range(4)))
+    student = run_bwd(dev, dL, causal, need=tuple(k == i2 for k in range(4)))
+    assert np.array_equal(teacher[i1], full[i1])
+    assert np.array_equal(student[i2], full[i2])
 
 
 def test_bwd_explicit_scales(orc):
@@ -205,7 +227,7 @@ def test_bwd_full_size_workload(orc):
     (dQ1, dK1, dQ2, dK2), fwd_out = run_bwd(dev, dL, True, saved=True)
     bits = oracle_bits(ins)
     rows = sample_rows(w.BH, w.NQ, 256, seed=w.seed)
-    oL, oA, oB, oq1, oq2 = orc.bwd_rows(*bits, rows, np.full(len(rows), g), causal=True)
+    oL, oA, oB, oq1, oq2 = fwdbwd16k_oracle(orc, bits, "rows", tuple(rows.ravel().tolist()), g)
     # the saved state the backward consumed: L, LSE1, LSE2 of the same rows
     check_fwd(fwd_out, (oL, oA, oB), rows, "fwdbwd16k forward")
     gq1 = dQ1.reshape(w.BH, w.NQ, -1)[rows[:, 0], rows[:, 1]]
@@ -213,7 +235,7 @@ def test_bwd_full_size_workload(orc):
     assert rel_frobenius(gq1, oq1) <= TOL_GRAD
     assert rel_frobenius(gq2, oq2) <= TOL_GRAD
     heads = [0, int(np.random.default_rng(w.seed).integers(1, w.BH))]
-    o = orc.bwd_heads(*bits, heads, np.full((2, w.NQ), g), causal=True)
+    o = fwdbwd16k_oracle(orc, bits, "heads", tuple(heads), g)
     for n, G in (("dK1", dK1), ("dK2", dK2)):
         err = rel_frobenius(G.reshape(w.BH, w.NK, -1)[heads], o[n])
         assert err <= TOL_GRAD, f"{n} {err:.3e}"
@@ -228,10 +250,8 @@ def test_bwd_full_size_one_sided(orc, bwd_algo, side):
     """The one-sided kernels on the forward+backward workload (B1 H32 N16384 d128
     causal): the student side alone (the page's configuration 1, standard
     distillation) or the teacher side alone; dQ on sampled rows of every head,
-    dK in full on head 0 and one seeded head.  The specialised kernels are the
-    fused path's; the split path is covered at this size by the test above."""
-    if bwd_algo != "fused":
-        pytest.skip("the one-sided kernels are the fused path")
+    dK in full on head 0 and one seeded head.  Every algorithm has instances
+    specialised to one side."""
     from attention_kl_distillation_b200.inputs import WORKLOADS, make_inputs, sample_rows
     w = WORKLOADS["fwdbwd16k"]
     ins = make_inputs(w)
@@ -244,10 +264,10 @@ def test_bwd_full_size_one_sided(orc, bwd_algo, side):
     assert all(out[i] is None for i in range(4) if not need[i])
     bits = oracle_bits(ins)
     rows = sample_rows(w.BH, w.NQ, 256, seed=w.seed + 1)
-    _, _, _, oq1, oq2 = orc.bwd_rows(*bits, rows, np.full(len(rows), g), causal=True)
+    _, _, _, oq1, oq2 = fwdbwd16k_oracle(orc, bits, "rows", tuple(rows.ravel().tolist()), g)
     gq = dQ.reshape(w.BH, w.NQ, -1)[rows[:, 0], rows[:, 1]]
     assert rel_frobenius(gq, oq2 if side == "student" else oq1) <= TOL_GRAD
     heads = [0, int(np.random.default_rng(w.seed + 1).integers(1, w.BH))]
-    o = orc.bwd_heads(*bits, heads, np.full((2, w.NQ), g), causal=True)
+    o = fwdbwd16k_oracle(orc, bits, "heads", tuple(heads), g)
     err = rel_frobenius(dK.reshape(w.BH, w.NK, -1)[heads], o["dK2" if side == "student" else "dK1"])
     assert err <= TOL_GRAD, f"{side} dK {err:.3e}"
