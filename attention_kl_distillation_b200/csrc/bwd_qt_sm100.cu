@@ -38,7 +38,10 @@
 //               the fp32 workspace with coalesced reductions; at the end of a
 //               unit converts the dQ accumulators to bf16 and stores them.
 // TMEM (512 columns): S1 [0,64) S2 [64,128) dQ1 [128,128+d1) dQ2 [..,+d2)
-//                     dK1^T [384,448) dK2^T [448,512).
+//                     dK1^T [384,448) dK2^T [448,512).  A one-sided instance
+//                     keeps its side's dQ from column 128 and a second S buffer
+//                     after it, so S of step t+1 need not wait for the dS warps
+//                     to read S of step t.
 //
 // Gradient sets as in the key-tile kernel: SEL = 1 (teacher side), 2 (student
 // side), 3 (both); a one-sided instance forms and contracts only its own dS,
@@ -88,9 +91,9 @@ struct QtLayout {  // NDT: dS tiles per buffer (1 or 2 gradient sides)
   static constexpr int k_off = q2_off + q2_bytes;
   static constexpr int ds_off = k_off + KSTAGES * kstage_bytes;
   static constexpr int bar_off = ds_off + DSBUF * NDT * ds_bytes;
-  // qfull qempty kfull[K] kempty[K] sfull sempty dsfull[D] dsempty[D] dkfull
-  // dkempty[2] dqfull dqempty ufull[2] uempty[2] drain
-  static constexpr int nbar = 2 + 2 * KSTAGES + 2 + 2 * DSBUF + 5 + 4 + 1;
+  // qfull qempty kfull[K] kempty[K] sfull[2] sempty[2] dsfull[D] dsempty[D]
+  // dkfull dkempty[2] dqfull dqempty ufull[2] uempty[2] drain
+  static constexpr int nbar = 2 + 2 * KSTAGES + 4 + 2 * DSBUF + 5 + 4 + 1;
   static constexpr int misc_off = bar_off + nbar * 8;
   static constexpr int total = misc_off + 32;
   static constexpr int alloc = total + 1024;
@@ -224,6 +227,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // dK accumulator row: the wanted sides only, teacher first
   constexpr int LDK = (G1 ? D1 : 0) + (G2 ? D2 : 0);
   constexpr int DK2_COL = G1 ? D1 : 0;
+  // dQ accumulators from column 128: dQ1 then dQ2, or the one side asked for.
+  // S buffers: one for both sides; two for one side, the second right after
+  // that side's dQ (at most [256, 384), below dK1^T).
+  constexpr uint32_t kColDQ2 = G1 ? kColDQ1 + D1 : kColDQ1;
+  constexpr int NSB = (G1 && G2) ? 1 : 2;
+  constexpr uint32_t kColSB1 = kColDQ1 + (G1 ? D1 : 0) + (G2 ? D2 : 0);
+  static_assert(NSB == 1 || kColSB1 + 128 <= kColDK1, "TMEM budget exceeded");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -232,9 +242,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* qempty = bars + 1;
   uint64_t* kfull = bars + 2;
   uint64_t* kempty = kfull + KST;
-  uint64_t* sfull = kempty + KST;
-  uint64_t* sempty = sfull + 1;
-  uint64_t* dsfull = sempty + 1;
+  uint64_t* sfull = kempty + KST;  // [2]
+  uint64_t* sempty = sfull + 2;    // [2]
+  uint64_t* dsfull = sempty + 2;
   uint64_t* dsempty = dsfull + DSB;
   uint64_t* dkfull = dsempty + DSB;
   uint64_t* dkempty = dkfull + 1;  // [2]: dK1^T and dK2^T slots read out
@@ -259,8 +269,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&kfull[s], 1);
       mbar_init(&kempty[s], 1);
     }
-    mbar_init(sfull, 1);
-    mbar_init(sempty, 4 * NDS);  // every warp of every dS warpgroup
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 4 * NDS);  // every warp of every dS warpgroup
+    }
     for (int s = 0; s < DSB; ++s) {
       mbar_init(&dsfull[s], 4 * NDS);
       mbar_init(&dsempty[s], 1);
@@ -369,8 +381,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint64_t q1d = sdesc_sw128(q1a, 16, 1024), q2d = sdesc_sw128(q2a, 16, 1024);
       // Q tiles read MN-major for dK^T: 64-feature chunks 16 KB apart
       const uint64_t q1m = sdesc_sw128(q1a, RQ * 128, 1024), q2m = sdesc_sw128(q2a, RQ * 128, 1024);
-      int us = 0, ks_s = 0, ks_r = 0, db = 0;
-      uint32_t uph = 0, qph = 0, kph_s = 0, sph = 0, dqph = 0;
+      int us = 0, ks_s = 0, ks_r = 0, db = 0, sb = 0;
+      uint32_t uph = 0, qph = 0, kph_s = 0, dqph = 0;
+      uint32_t sph = 0;  // bit b: parity of S buffer b's current use
       uint32_t dkph[2] = {0, 0};
       uint32_t dsph[DSB] = {};
       bool ok = true;
@@ -388,24 +401,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         qph ^= 1;
         auto issue_s = [&]() -> bool {
           if (!mbar_wait(&kfull[ks_s], kph_s, ctl)) return false;
-          if (!mbar_wait(sempty, sph ^ 1, ctl)) return false;
+          if (!mbar_wait(&sempty[sb], ((sph >> sb) & 1u) ^ 1u, ctl)) return false;
           tc_fence_after();
+          const uint32_t scol = tmem_base + (sb == 0 ? 0u : kColSB1);
           const uint64_t k1d = sdesc_sw128(smem_u32(k1_s(ks_s)), 16, 1024);
           const uint64_t k2d = sdesc_sw128(smem_u32(k2_s(ks_s)), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D1 / 16; ++kk) {
             const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(tmem_base + kColS1, sdesc_advance(q1d, (kk >> 2) * (RQ * 128) + o),
+            umma_bf16_ss(scol + kColS1, sdesc_advance(q1d, (kk >> 2) * (RQ * 128) + o),
                          sdesc_advance(k1d, (kk >> 2) * (CK * 128) + o), idS, kk > 0);
           }
 #pragma unroll
           for (int kk = 0; kk < D2 / 16; ++kk) {
             const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(tmem_base + kColS2, sdesc_advance(q2d, (kk >> 2) * (RQ * 128) + o),
+            umma_bf16_ss(scol + kColS2, sdesc_advance(q2d, (kk >> 2) * (RQ * 128) + o),
                          sdesc_advance(k2d, (kk >> 2) * (CK * 128) + o), idS, kk > 0);
           }
-          umma_commit(sfull);
-          sph ^= 1;
+          umma_commit(&sfull[sb]);
+          sph ^= 1u << sb;
+          if (NSB == 2) sb ^= 1;
           if (++ks_s == KST) {
             ks_s = 0;
             kph_s ^= 1;
@@ -431,7 +446,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                            sdesc_sw128(smem_u32(k1_s(ks_r)) + kk * 2048, CK * 128, 1024), idQ1,
                            (t > 0 || kk > 0));
             if (G2 && p.want_dq2)
-              umma_bf16_ss(tmem_base + kColDQ1 + D1,
+              umma_bf16_ss(tmem_base + kColDQ2,
                            sdesc_sw128(smem_u32(ds2_s(db)) + kk * 32, 16, 1024),
                            sdesc_sw128(smem_u32(k2_s(ks_r)) + kk * 2048, CK * 128, 1024), idQ2,
                            (t > 0 || kk > 0));
@@ -483,8 +498,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row within the tile
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    int us = 0, db = 0;
-    uint32_t uph = 0, sph = 0;
+    int us = 0, db = 0, sb = 0;
+    uint32_t uph = 0;
+    uint32_t sph = 0;  // bit b: parity of S buffer b's current use
     uint32_t dsph[DSB] = {};
     bool ok = true;
     for (;;) {
@@ -515,18 +531,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int t = 0; t < w.nsteps; ++t) {
         const int ks = w.step(t);
         const int k0 = ks * CK;
-        if (!(ok = mbar_wait(sfull, sph, ctl))) break;
-        sph ^= 1;
+        if (!(ok = mbar_wait(&sfull[sb], (sph >> sb) & 1u, ctl))) break;
+        sph ^= 1u << sb;
         tc_fence_after();
+        const uint32_t scol = tl + (sb == 0 ? 0u : kColSB1);
         uint32_t a[KPW], b[KPW];
-        tmem_ld_32x32b<KPW>(tl + kColS1 + part * KPW, a);
-        tmem_ld_32x32b<KPW>(tl + kColS2 + part * KPW, b);
+        tmem_ld_32x32b<KPW>(scol + kColS1 + part * KPW, a);
+        tmem_ld_32x32b<KPW>(scol + kColS2 + part * KPW, b);
         tmem_ld_wait();
         reg_fence(a);
         reg_fence(b);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(sempty);
+        if (lane == 0) mbar_arrive(&sempty[sb]);
+        if (NSB == 2) sb ^= 1;
         const bool masked = ks >= w.kmask;
         const int last = lim - k0;
         const uint32_t r1 = smem_u32(ds1_s(db)) + rowoff, r2 = smem_u32(ds2_s(db)) + rowoff;
@@ -629,7 +647,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int D = tsel == 0 ? D1 : D2;
         __nv_bfloat16* dst =
             (tsel == 0 ? p.dQ1 : p.dQ2) + (static_cast<size_t>(w.bh) * p.NQ + i) * D;
-        const uint32_t col0 = tl + kColDQ1 + (tsel == 0 ? 0 : D1);
+        const uint32_t col0 = tl + (tsel == 0 ? kColDQ1 : kColDQ2);
 #pragma unroll
         for (int c = 0; c < DMAX; c += 32) {
           if (c >= D) break;

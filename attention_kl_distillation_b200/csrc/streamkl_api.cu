@@ -196,12 +196,13 @@ int bwd_algo_setting() {
   return v;
 }
 
-// AUTO: the page keeps the fused kernel while its dQ reductions stay cheap and
-// switches to separate kernels when they contend.  On B200 the fused kernel
-// measured faster up to the largest accumulator tested (B1 H32 N16384 d128:
-// 537 MB of fp32 dQ, fused 9.9 ms vs split 10.7 ms), so the threshold sits
-// above every measured shape; set the algorithm explicitly to override.
-constexpr size_t kFusedDqAccLimit = 4ull << 30;
+// AUTO: the page keeps the fused kernel while its atomic reductions stay cheap
+// and switches to separate kernels when they contend.  On B200 the fused
+// kernels measured faster at every size tested, in or beyond L2: B1 H32 N16384
+// d128 causal (537 MB fp32 accumulator) fused query tiles 8.17 ms, fused key
+// tiles 9.43, split 10.37; B1 H80 N65536 d128 causal (5 GiB accumulator)
+// 357, 365 and 400 ms (bench.py --compare-bwd).  So AUTO is FUSED at every
+// size; SPLIT stays available explicitly.
 
 // SMs of the current device for scheduling decisions; 148 (B200) when no
 // device can be queried, so that the decision is the same on a host without one.
@@ -230,10 +231,7 @@ streamkl_bwd_algorithm resolve_bwd_algo(const streamkl_problem& pr) {
   if (a == STREAMKL_BWD_SPLIT || a == STREAMKL_BWD_FUSED_KEY_TILES ||
       a == STREAMKL_BWD_FUSED_QUERY_TILES)
     return static_cast<streamkl_bwd_algorithm>(a);
-  if (a == STREAMKL_BWD_FUSED) return fused_orientation(pr);
-  const size_t acc = static_cast<size_t>(pr.B) * pr.H * static_cast<size_t>(pr.NQ) *
-                     static_cast<size_t>(pr.d1 + pr.d2) * sizeof(float);
-  return acc > kFusedDqAccLimit ? STREAMKL_BWD_SPLIT : fused_orientation(pr);
+  return fused_orientation(pr);  // FUSED and AUTO
 }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }

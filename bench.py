@@ -70,6 +70,10 @@ def parse_args(argv=None):
     ap.add_argument("--bwd-algo", default="auto",
                     choices=["auto", "fused", "split", "fused_key_tiles", "fused_query_tiles"],
                     help="streamkl_bwd algorithm (process-wide setting of the library)")
+    ap.add_argument("--compare-bwd", action="store_true",
+                    help="instead of the bench line, one JSON line per backward algorithm on the "
+                         "workload (median of --steps calls after --warmup): the measurement the "
+                         "library's AUTO selection rests on")
     ap.add_argument("--need", default="1111",
                     help="which of dQ1 dK1 dQ2 dK2 the backward returns (e.g. 0101 = dK only)")
     return ap.parse_args(argv)
@@ -374,6 +378,45 @@ def run_table(args):
         torch.cuda.empty_cache()
 
 
+def run_compare_bwd(args, w: Workload):
+    """Times streamkl_bwd with each algorithm on one workload (same inputs, same saved
+    state), so that the fused/split choice can be set from a measurement."""
+    import attention_kl_distillation_b200 as skl
+    from attention_kl_distillation_b200 import binding
+    peak, _, _ = peaks()
+    dev = torch.device("cuda", 0)
+    Q1, K1, Q2, K2 = (t.to(dev) for t in make_inputs(w))
+    L, A, B = skl.fwd(Q1, K1, Q2, K2, causal=w.causal)
+    dL = torch.full((w.B, w.H, w.NQ), 1.0 / (w.B * w.H * w.NQ), device=dev)
+    grads = tuple(torch.empty_like(t) for t in (Q1, K1, Q2, K2))
+    ws = torch.empty(binding.workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal),
+                     dtype=torch.uint8, device=dev)
+    acc_bytes = w.BH * w.NQ * (w.d1 + w.d2) * 4
+    for algo in ("fused_query_tiles", "fused_key_tiles", "split"):
+        binding.set_bwd_algorithm(algo)
+        for _ in range(max(1, args.warmup)):
+            skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal, workspace=ws, out=grads)
+        times = []
+        for _ in range(max(1, args.steps)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal, workspace=ws, out=grads)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        if skl.query_device_status() != 0:
+            raise RuntimeError("device status reported an error")
+        ms = statistics.median(times)
+        tf = w.bwd_flops() / (ms * 1e-3) / 1e12
+        print(json.dumps({"workload": workload_desc(w, "fwdbwd")["workload"], "algorithm": algo,
+                          "calls": len(times), "median_ms": ms, "tflops": tf,
+                          "frac_of_measured_bf16": tf / peak,
+                          "fp32_accumulator_bytes": acc_bytes}), flush=True)
+    binding.set_bwd_algorithm("auto")
+    print(json.dumps({"auto_selects": binding.bwd_algorithm_for(w.B, w.H, w.NQ, w.NK, w.d1, w.d2,
+                                                                w.causal)}), flush=True)
+
+
 # --------------------------------------------------------------------------- our path
 def main(argv=None):
     args = parse_args(argv)
@@ -387,6 +430,8 @@ def main(argv=None):
     phase = args.phase if args.phase != "auto" else ("fwdbwd" if w.backward else "fwd")
     if args.impl == "reference":
         return run_reference(args, w, phase)
+    if args.compare_bwd:
+        return run_compare_bwd(args, w)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
