@@ -84,16 +84,16 @@ struct QtLayout {  // NDT: dS tiles per buffer (1 or 2 gradient sides)
   static constexpr bool fits(int k, int d) {
     return fixed_bytes + k * kstage_bytes + d * NDT * ds_bytes <= 232448;
   }
-  static constexpr int DSBUF = 1;
+  static constexpr int DSBUF = 1;  // the dS warps' store waits on the previous step's kempty
   static constexpr int KSTAGES = fits(4, DSBUF) ? 4 : 3;
   static constexpr int q1_off = 0;
   static constexpr int q2_off = q1_off + q1_bytes;
   static constexpr int k_off = q2_off + q2_bytes;
   static constexpr int ds_off = k_off + KSTAGES * kstage_bytes;
   static constexpr int bar_off = ds_off + DSBUF * NDT * ds_bytes;
-  // qfull qempty kfull[K] kempty[K] sfull[2] sempty[2] dsfull[D] dsempty[D]
-  // dkfull dkempty[2] dqfull dqempty ufull[2] uempty[2] drain
-  static constexpr int nbar = 2 + 2 * KSTAGES + 4 + 2 * DSBUF + 5 + 4 + 1;
+  // qfull qempty kfull[K] kempty[K] sfull[2] sempty[2] dsfull[D] dkempty[2]
+  // dqfull dqempty ufull[2] uempty[2] drain
+  static constexpr int nbar = 2 + 2 * KSTAGES + 4 + DSBUF + 4 + 4 + 1;
   static constexpr int misc_off = bar_off + nbar * 8;
   static constexpr int total = misc_off + 32;
   static constexpr int alloc = total + 1024;
@@ -244,10 +244,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* kempty = kfull + KST;
   uint64_t* sfull = kempty + KST;  // [2]
   uint64_t* sempty = sfull + 2;    // [2]
+  // kempty[s] completes when the products of the step that used key stage s
+  // are done: the producer may refill the stage, the dS buffer of that step is
+  // free again and its dK^T is in TMEM.  One commit per step serves all three.
   uint64_t* dsfull = sempty + 2;
-  uint64_t* dsempty = dsfull + DSB;
-  uint64_t* dkfull = dsempty + DSB;
-  uint64_t* dkempty = dkfull + 1;  // [2]: dK1^T and dK2^T slots read out
+  uint64_t* dkempty = dsfull + DSB;  // [2]: dK1^T and dK2^T slots read out
   uint64_t* dqfull = dkempty + 2;
   uint64_t* dqempty = dqfull + 1;
   uint64_t* ufull = dqempty + 1;
@@ -273,11 +274,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&sfull[s], 1);
       mbar_init(&sempty[s], 4 * NDS);  // every warp of every dS warpgroup
     }
-    for (int s = 0; s < DSB; ++s) {
-      mbar_init(&dsfull[s], 4 * NDS);
-      mbar_init(&dsempty[s], 1);
-    }
-    mbar_init(dkfull, 1);
+    for (int s = 0; s < DSB; ++s) mbar_init(&dsfull[s], 4 * NDS);
     mbar_init(&dkempty[0], 4);
     mbar_init(&dkempty[1], 4);
     mbar_init(dqfull, 1);
@@ -437,24 +434,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             dqph ^= 1;
           }
           tc_fence_after();
+          // Descriptors of this step's operands are built once; each UMMA below
+          // adds a constant offset.  The single issuing thread needs about as long
+          // to issue an M128 N64 product as the tensor pipe takes to run an N128
+          // one, so little else may sit between the issues.
+          const uint32_t ds1a = smem_u32(ds1_s(db)), ds2a = smem_u32(ds2_s(db));
+          const uint64_t d1k = sdesc_sw128(ds1a, 16, 1024), d2k = sdesc_sw128(ds2a, 16, 1024);
+          const uint64_t d1m = sdesc_sw128(ds1a, CK * 128, 1024), d2m = sdesc_sw128(ds2a, CK * 128, 1024);
+          const uint64_t k1m = sdesc_sw128(smem_u32(k1_s(ks_r)), CK * 128, 1024);
+          const uint64_t k2m = sdesc_sw128(smem_u32(k2_s(ks_r)), CK * 128, 1024);
+          const uint32_t acc0 = t > 0;
           // dQ_t += (s_t dS_t) K_t : A = dS (K-major, 128B rows of 64 keys), B = K_t
           // read MN-major (features contiguous; 64-feature chunks 8 KB apart).
+          if (G1 && p.want_dq1) {
 #pragma unroll
-          for (int kk = 0; kk < CK / 16; ++kk) {
-            if (G1 && p.want_dq1)
-              umma_bf16_ss(tmem_base + kColDQ1, sdesc_sw128(smem_u32(ds1_s(db)) + kk * 32, 16, 1024),
-                           sdesc_sw128(smem_u32(k1_s(ks_r)) + kk * 2048, CK * 128, 1024), idQ1,
-                           (t > 0 || kk > 0));
-            if (G2 && p.want_dq2)
-              umma_bf16_ss(tmem_base + kColDQ2,
-                           sdesc_sw128(smem_u32(ds2_s(db)) + kk * 32, 16, 1024),
-                           sdesc_sw128(smem_u32(k2_s(ks_r)) + kk * 2048, CK * 128, 1024), idQ2,
-                           (t > 0 || kk > 0));
+            for (int kk = 0; kk < CK / 16; ++kk)
+              umma_bf16_ss(tmem_base + kColDQ1, sdesc_advance(d1k, kk * 32),
+                           sdesc_advance(k1m, kk * 2048), idQ1, kk > 0 ? 1u : acc0);
+          }
+          if (G2 && p.want_dq2) {
+#pragma unroll
+            for (int kk = 0; kk < CK / 16; ++kk)
+              umma_bf16_ss(tmem_base + kColDQ2, sdesc_advance(d2k, kk * 32),
+                           sdesc_advance(k2m, kk * 2048), idQ2, kk > 0 ? 1u : acc0);
           }
           // dK_t^T = Q_t^T (s_t dS_t) : A = Q tile read MN-major (64-feature chunks
           // 16 KB apart), B = dS read MN-major (64 keys contiguous per query).
-          const uint64_t d1m = sdesc_sw128(smem_u32(ds1_s(db)), CK * 128, 1024);
-          const uint64_t d2m = sdesc_sw128(smem_u32(ds2_s(db)), CK * 128, 1024);
           if (G1) {
             if (!(ok = mbar_wait(&dkempty[0], dkph[0] ^ 1, ctl))) break;
             dkph[0] ^= 1;
@@ -477,9 +482,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                              sdesc_advance(d2m, kk * 2048), idK2, kk > 0);
             }
           }
-          umma_commit(dkfull);
-          umma_commit(&dsempty[db]);
-          umma_commit(&kempty[ks_r]);
+          umma_commit(&kempty[ks_r]);  // step done: K stage free, dS buffer free, dK^T ready
           if (++db == DSB) db = 0;
           if (++ks_r == KST) ks_r = 0;
         }
@@ -501,7 +504,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int us = 0, db = 0, sb = 0;
     uint32_t uph = 0;
     uint32_t sph = 0;  // bit b: parity of S buffer b's current use
-    uint32_t dsph[DSB] = {};
+    int pks = -1;        // K stage of the previous step (-1: none yet)
+    uint32_t pkph = 0;   // its phase
+    int cks = 0;         // K stage of the current step
+    uint32_t ckph = 0;
     bool ok = true;
     for (;;) {
       if (!(ok = mbar_wait(&ufull[us], uph, ctl))) break;
@@ -550,15 +556,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t r1 = smem_u32(ds1_s(db)) + rowoff, r2 = smem_u32(ds2_s(db)) + rowoff;
         // dS is formed in registers first, with the whole segment's arithmetic
         // in flight at once, while the previous step's contractions may still
-        // read the buffer; it is stored once they are done.
+        // read the buffer; it is stored once they are done (the previous
+        // step's key stage released).
         uint32_t w1[KPW / 2], w2[KPW / 2];
         if (masked)
           form_ds_regs<true, G1, G2>(a, b, rr, p.c1, p.c2, last, w1, w2);
         else
           form_ds_regs<false, G1, G2>(a, b, rr, p.c1, p.c2, 0, w1, w2);
-        if (!(ok = mbar_wait(&dsempty[db], dsph[db] ^ 1, ctl))) break;
-        dsph[db] ^= 1;
+        if (pks >= 0 && !(ok = mbar_wait(&kempty[pks], pkph, ctl))) break;
         store_ds<G1, G2>(w1, w2, r, part * (KPW / 8), r1, r2);
+        pks = cks;
+        pkph = ckph;
+        if (++cks == KST) {
+          cks = 0;
+          ckph ^= 1;
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&dsfull[db]);
@@ -575,7 +587,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int f1 = (D1 == 128) ? quarter * 32 + lane : (lane < 16 ? quarter * 16 + lane : -1);
     const int f2 = (D2 == 128) ? quarter * 32 + lane : (lane < 16 ? quarter * 16 + lane : -1);
     int us = 0;
-    uint32_t uph = 0, dkph = 0, dqph = 0;
+    uint32_t uph = 0, dqph = 0;
+    int cks = 0;
+    uint32_t ckph = 0;
     bool ok = true;
     for (;;) {
       if (!(ok = mbar_wait(&ufull[us], uph, ctl))) break;
@@ -590,8 +604,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const UnitQ w = decode_unit(p, u);
       for (int t = 0; t < w.nsteps; ++t) {
         const int k0 = w.step(t) * CK;
-        if (!(ok = mbar_wait(dkfull, dkph, ctl))) break;
-        dkph ^= 1;
+        if (!(ok = mbar_wait(&kempty[cks], ckph, ctl))) break;
+        if (++cks == KST) {
+          cks = 0;
+          ckph ^= 1;
+        }
         tc_fence_after();
         const int nvalid = min(CK, p.NK - k0);
         float* base = p.dKacc + (static_cast<size_t>(w.bh) * p.NK + k0) * LDK;
