@@ -93,12 +93,13 @@ def launch_count() -> int:
     return int(_lib.streamkl_launch_count())
 
 
-BWD_ALGOS = {"auto": 0, "fused": 1, "split": 2, "fused_key_tiles": 3, "fused_query_tiles": 4}
+BWD_ALGOS = {"auto": 0, "fused": 1, "split": 2, "fused_key_tiles": 3, "fused_query_tiles": 4,
+             "fused_sides": 5}
 
 
 def set_bwd_algorithm(name: str) -> None:
-    """Process-wide backward algorithm: "auto", "fused", "split", "fused_key_tiles" or
-    "fused_query_tiles" (see streamkl_bwd_algorithm in include/streamkl.h)."""
+    """Process-wide backward algorithm: "auto", "fused", "split", "fused_key_tiles",
+    "fused_query_tiles" or "fused_sides" (see streamkl_bwd_algorithm in include/streamkl.h)."""
     st = _lib.streamkl_set_bwd_algorithm(BWD_ALGOS[name])
     if st != OK:
         raise StreamKLError(st, "streamkl_set_bwd_algorithm")

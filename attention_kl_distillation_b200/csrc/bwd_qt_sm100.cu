@@ -619,27 +619,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int f = tsel == 0 ? f1 : DK2_COL + f2;
           const bool fok = (tsel == 0 ? f1 : f2) >= 0;
           const uint32_t col = tl + (tsel == 0 ? kColDK1 : kColDK2);
-          // two halves of 32 keys; the slot is released once both are in registers
+          // both halves of 32 keys into registers, the slot released, then the reductions
           uint32_t v0[32], v1[32];
           if (want) {
             tmem_ld_32x32b_x32(col, v0);
+            tmem_ld_32x32b_x32(col + 32, v1);
             tmem_ld_wait();
             reg_fence(v0);
+            reg_fence(v1);
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dkempty[tsel]);
           if (want && fok) {
             if (nvalid == CK)
               red_dk<LDK, true>(base + f, v0, 32);
             else
               red_dk<LDK, false>(base + f, v0, nvalid);
           }
-          if (want) {
-            tmem_ld_32x32b_x32(col + 32, v1);
-            tmem_ld_wait();
-            reg_fence(v1);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&dkempty[tsel]);
           if (want && fok) {
             if (nvalid == CK)
               red_dk<LDK, true>(base + 32 * LDK + f, v1, 32);

@@ -134,6 +134,30 @@ struct BwdQtParams {
 // sel as for launch_bwd.
 cudaError_t launch_bwd_qt(const BwdQtParams& p, int d1, int d2, int sel, int grid,
                           cudaStream_t stream);
+
+// One gradient side per launch, 128-query units and 128-key steps (every
+// product N = 128): side 1 forms dS1 and writes dQ1 / reduces dK1, side 2 the
+// same for the student.  Both sides are two launches sharing the accumulator.
+struct BwdSideParams {
+  CUtensorMap tmQ1, tmK1, tmQ2, tmK2;  // 128-row boxes
+  const float* L;
+  const float* LSE1;
+  const float* LSE2;
+  const float* dL;
+  float* dKacc;         // [BH][NK][ldk] fp32, this side's columns from dk_col, zeroed first
+  int ldk, dk_col;
+  int* counter;         // work-unit counter of this launch, zeroed first
+  __nv_bfloat16* dQ;    // [BH][NQ][d_t] of this side, or null
+  int BH, NQ, NK, causal;
+  int want_dq, want_dk;
+  float c1, c2;  // s_t * log2(e)
+  float s1, s2;
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+cudaError_t launch_bwd_side(const BwdSideParams& p, int d1, int d2, int side, int grid,
+                            cudaStream_t stream);
 __host__ __device__ inline int bwd_qt_units(int BH, int NQ) {
   return BH * ((NQ + kBwdQtRows - 1) / kBwdQtRows);
 }

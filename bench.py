@@ -68,7 +68,8 @@ def parse_args(argv=None):
                     help="N > 1: every rank runs the whole workload (replicas, weak scaling) or "
                          "a contiguous range of its B*H heads (heads, strong scaling)")
     ap.add_argument("--bwd-algo", default="auto",
-                    choices=["auto", "fused", "split", "fused_key_tiles", "fused_query_tiles"],
+                    choices=["auto", "fused", "split", "fused_key_tiles", "fused_query_tiles",
+                             "fused_sides"],
                     help="streamkl_bwd algorithm (process-wide setting of the library)")
     ap.add_argument("--compare-bwd", action="store_true",
                     help="instead of the bench line, one JSON line per backward algorithm on the "
@@ -340,7 +341,7 @@ def run_table(args):
                           lambda: skl.fwd_splitk(Q1, K1, Q2, K2, causal=w.causal, nsplit=ns,
                                                  workspace=fws, out=(L, A, B)), w.fwd_flops()))
         if w.backward:
-            for algo in ("fused_key_tiles", "fused_query_tiles", "split"):
+            for algo in ("fused_key_tiles", "fused_query_tiles", "fused_sides", "split"):
                 calls.append((f"bwd_{algo}", algo,
                               lambda: skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal,
                                               workspace=ws, out=grads), w.bwd_flops()))
@@ -392,7 +393,7 @@ def run_compare_bwd(args, w: Workload):
     ws = torch.empty(binding.workspace_size(w.B, w.H, w.NQ, w.NK, w.d1, w.d2, w.causal),
                      dtype=torch.uint8, device=dev)
     acc_bytes = w.BH * w.NQ * (w.d1 + w.d2) * 4
-    for algo in ("fused_query_tiles", "fused_key_tiles", "split"):
+    for algo in ("fused_query_tiles", "fused_sides", "fused_key_tiles", "split"):
         binding.set_bwd_algorithm(algo)
         for _ in range(max(1, args.warmup)):
             skl.bwd(dL, Q1, K1, Q2, K2, L, A, B, causal=w.causal, workspace=ws, out=grads)

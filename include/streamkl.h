@@ -196,9 +196,13 @@ streamkl_status streamkl_bwd_noalloc(const streamkl_problem *prob, const float *
  *                     reductions.  Each dS thread then owns a query row, so
  *                     its L, LSE and dL are registers instead of shared-memory
  *                     loads for every key.
+ *  FUSED_SIDES        query-tile units with one gradient side per pass and
+ *                     128-key steps: every product is N = 128, both S
+ *                     products are recomputed once per side asked for.
  *  FUSED              the fused orientation chosen by shape: query tiles when
  *                     B*H*ceil(NQ/128) fills the device's SMs twice, else key
- *                     tiles.
+ *                     tiles; with query tiles and one side asked for,
+ *                     FUSED_SIDES (measured faster for one side).
  *  SPLIT              two passes of one kernel: a dK pass over key tiles and
  *                     a dQ pass over query tiles, each regenerating the
  *                     probabilities; no reductions in global memory.
@@ -216,13 +220,16 @@ typedef enum {
   STREAMKL_BWD_FUSED = 1,
   STREAMKL_BWD_SPLIT = 2,
   STREAMKL_BWD_FUSED_KEY_TILES = 3,
-  STREAMKL_BWD_FUSED_QUERY_TILES = 4
+  STREAMKL_BWD_FUSED_QUERY_TILES = 4,
+  STREAMKL_BWD_FUSED_SIDES = 5
 } streamkl_bwd_algorithm;
 
 streamkl_status streamkl_set_bwd_algorithm(streamkl_bwd_algorithm algo);
 
-/* The algorithm streamkl_bwd would use for this problem on the current device:
- * SPLIT, FUSED_KEY_TILES or FUSED_QUERY_TILES (AUTO and FUSED resolved). */
+/* The algorithm streamkl_bwd would use for this problem on the current device
+ * when both sides are asked for: SPLIT, FUSED_KEY_TILES, FUSED_QUERY_TILES or
+ * FUSED_SIDES (AUTO and FUSED resolved; for one side, FUSED_QUERY_TILES under
+ * AUTO or FUSED runs as FUSED_SIDES). */
 streamkl_bwd_algorithm streamkl_bwd_algorithm_for(const streamkl_problem *prob);
 
 /* Static English text for a status code. */

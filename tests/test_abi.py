@@ -114,7 +114,7 @@ def test_bwd_algorithm_selection():
     lib = B.lib()
     assert lib.streamkl_set_bwd_algorithm(7) == B.EINVAL
     try:
-        for name in ("split", "fused_key_tiles", "fused_query_tiles"):
+        for name in ("split", "fused_key_tiles", "fused_query_tiles", "fused_sides"):
             B.set_bwd_algorithm(name)
             assert B.bwd_algorithm_for(1, 2, 256, 256, 64, 64) == name
         B.set_bwd_algorithm("fused")

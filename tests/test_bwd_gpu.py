@@ -8,10 +8,11 @@ from gpu_common import TOL_GRAD, check_fwd, cuda_inputs, oracle_bits, rel_froben
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["fused_key_tiles", "fused_query_tiles", "split"])
+@pytest.fixture(autouse=True, params=["fused_key_tiles", "fused_query_tiles", "fused_sides", "split"])
 def bwd_algo(request):
     """Every backward test runs with each algorithm of streamkl_bwd: the fused kernel
-    with key-tile units and with query-tile units, and the two split passes."""
+    with key-tile units, with query-tile units, with query-tile units and one gradient
+    side per pass, and the two split passes."""
     from attention_kl_distillation_b200 import set_bwd_algorithm
     set_bwd_algorithm(request.param)
     yield request.param
