@@ -16,9 +16,10 @@
 //
 // B200 mapping (one CTA per SM, persistent, units handed out dynamically):
 //   work unit   (bh, 128-query tile); inner loop over the 128-key steps it sees
-//   warp 0      TMA producer: Q1/Q2 tile per unit, K1/K2 tiles per step into a
-//               ring whose K1 and K2 halves are freed separately (the other
-//               side's half once S is done, this side's once the step is done)
+//   warp 0      TMA producer: Q1/Q2 tile per unit, per step the keys of this
+//               side (K_t, read by S and dQ_t, free once the step is done) into
+//               a ring of up to four stages and the other side's keys (read by
+//               S only, free once S is done) into a shorter ring
 //   warp 1      TMEM owner and UMMA issuer, per step:
 //                 S1 = Q1 K1^T, S2 = Q2 K2^T                (M=128, N=128 keys)
 //                 dQ_t += dS_t K_t                          (M=128, N=d_t)
@@ -51,32 +52,40 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS1 = 0, kColS2 = 128, kColDQ = 256, kColDK = 384;
 
-template <int D1, int D2>
+template <int D1, int D2, int SIDE>
 struct SideLayout {
+  static constexpr int DT = SIDE == 1 ? D1 : D2;  // this side's head dimension
+  static constexpr int DO = SIDE == 1 ? D2 : D1;  // the other side's
   static constexpr int q1_bytes = RQ * D1 * 2;
   static constexpr int q2_bytes = RQ * D2 * 2;
-  static constexpr int k1_bytes = CK * D1 * 2;
-  static constexpr int k2_bytes = CK * D2 * 2;
-  static constexpr int kstage_bytes = k1_bytes + k2_bytes;
+  static constexpr int kt_bytes = CK * DT * 2;    // one stage of this side's keys
+  static constexpr int ko_bytes = CK * DO * 2;    // one stage of the other side's keys
   static constexpr int ds_bytes = RQ * CK * 2;  // dS_t, bf16 [128 queries][128 keys], two 64-key chunks
   static constexpr int fixed_bytes = q1_bytes + q2_bytes + ds_bytes + 1024 + 512;
-  static constexpr int ks_fit = (232448 - fixed_bytes) / kstage_bytes;
-  static constexpr int KSTAGES = ks_fit > 4 ? 4 : ks_fit;
+  static constexpr bool fits(int nt, int no) {
+    return fixed_bytes + nt * kt_bytes + no * ko_bytes <= 232448;
+  }
+  // This side's keys stay from S of a step to its contractions, so their ring
+  // is the deeper one: the stage for step t+1 was freed by step t-2.  The other
+  // side's keys are free once S is done.
+  static constexpr int NO = fits(3, 2) ? 2 : 1;
+  static constexpr int NT = fits(4, NO) ? 4 : 3;
   static constexpr int q1_off = 0;
   static constexpr int q2_off = q1_off + q1_bytes;
   static constexpr int ds_off = q2_off + q2_bytes;
-  static constexpr int k_off = ds_off + ds_bytes;
-  static constexpr int bar_off = k_off + KSTAGES * kstage_bytes;
-  // qfull qempty kfull1[K] kfull2[K] kempty1[K] kempty2[K] sfull sempty dsfull dkempty
-  // dqfull dqempty ufull[2] uempty[2] drain
-  static constexpr int nbar = 2 + 4 * KSTAGES + 4 + 2 + 4 + 1;
+  static constexpr int kt_off = ds_off + ds_bytes;
+  static constexpr int ko_off = kt_off + NT * kt_bytes;
+  static constexpr int bar_off = ko_off + NO * ko_bytes;
+  // qfull qempty kfullT[NT] kemptyT[NT] kfullO[NO] kemptyO[NO] sfull sempty dsfull
+  // dkempty dqfull dqempty ufull[2] uempty[2] drain
+  static constexpr int nbar = 2 + 2 * NT + 2 * NO + 4 + 2 + 4 + 1;
   static constexpr int misc_off = bar_off + nbar * 8;
   static constexpr int total = misc_off + 32;
   static constexpr int alloc = total + 1024;
-  static_assert(KSTAGES >= 2, "key ring too shallow");
+  static_assert(fits(NT, NO), "key rings too deep");
   static_assert(alloc <= 232448, "shared memory budget exceeded");
-  static_assert(q1_bytes % 1024 == 0 && q2_bytes % 1024 == 0 && k1_bytes % 1024 == 0 &&
-                    k2_bytes % 1024 == 0,
+  static_assert(q1_bytes % 1024 == 0 && q2_bytes % 1024 == 0 && kt_bytes % 1024 == 0 &&
+                    ko_bytes % 1024 == 0,
                 "operand tiles must stay 1024-byte aligned");
 };
 
@@ -171,19 +180,20 @@ template <int D1, int D2, int SIDE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     streamkl_bwd_side_kernel(const __grid_constant__ BwdSideParams p) {
   constexpr int DT = SIDE == 1 ? D1 : D2;
-  using Lay = SideLayout<D1, D2>;
-  constexpr int KST = Lay::KSTAGES;
+  constexpr int DO = SIDE == 1 ? D2 : D1;
+  using Lay = SideLayout<D1, D2, SIDE>;
+  constexpr int NT = Lay::NT, NO = Lay::NO;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off);
   uint64_t* qfull = bars + 0;
   uint64_t* qempty = bars + 1;
-  uint64_t* kfull1 = bars + 2;         // [KST]
-  uint64_t* kfull2 = kfull1 + KST;     // [KST]
-  uint64_t* kempty1 = kfull2 + KST;    // [KST]
-  uint64_t* kempty2 = kempty1 + KST;   // [KST]
-  uint64_t* sfull = kempty2 + KST;
+  uint64_t* kfullT = bars + 2;        // [NT] this side's keys
+  uint64_t* kemptyT = kfullT + NT;    // [NT] completes when the step's products are done
+  uint64_t* kfullO = kemptyT + NT;    // [NO] the other side's keys
+  uint64_t* kemptyO = kfullO + NO;    // [NO] completes when S is done
+  uint64_t* sfull = kemptyO + NO;
   uint64_t* sempty = sfull + 1;
   uint64_t* dsfull = sempty + 1;
   uint64_t* dkempty = dsfull + 1;
@@ -192,10 +202,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* ufull = dqempty + 1;   // [2]
   uint64_t* uempty = ufull + 2;    // [2]
   uint64_t* drain = uempty + 2;
-  // this side's key half is released when the step's products are done; the
-  // other side's half when S is
-  uint64_t* kemptyT = SIDE == 1 ? kempty1 : kempty2;
-  uint64_t* kemptyO = SIDE == 1 ? kempty2 : kempty1;
+  const CUtensorMap* tmKT = SIDE == 1 ? &p.tmK1 : &p.tmK2;
+  const CUtensorMap* tmKO = SIDE == 1 ? &p.tmK2 : &p.tmK1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::misc_off + 4);
   volatile int* unit_slot = reinterpret_cast<volatile int*>(smem + Lay::misc_off + 8);  // [2]
@@ -208,11 +216,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     *abort_flag = 0;
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
-    for (int s = 0; s < KST; ++s) {
-      mbar_init(&kfull1[s], 1);
-      mbar_init(&kfull2[s], 1);
-      mbar_init(&kempty1[s], 1);
-      mbar_init(&kempty2[s], 1);
+    for (int s = 0; s < NT; ++s) {
+      mbar_init(&kfullT[s], 1);
+      mbar_init(&kemptyT[s], 1);
+    }
+    for (int s = 0; s < NO; ++s) {
+      mbar_init(&kfullO[s], 1);
+      mbar_init(&kemptyO[s], 1);
     }
     mbar_init(sfull, 1);
     mbar_init(sempty, 4 * NDS);
@@ -244,16 +254,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* q1_s = smem + Lay::q1_off;
   uint8_t* q2_s = smem + Lay::q2_off;
   uint8_t* ds_s = smem + Lay::ds_off;
-  auto k1_s = [&](int s) { return smem + Lay::k_off + s * Lay::kstage_bytes; };
-  auto k2_s = [&](int s) { return smem + Lay::k_off + s * Lay::kstage_bytes + Lay::k1_bytes; };
+  auto kt_s = [&](int s) { return smem + Lay::kt_off + s * Lay::kt_bytes; };
+  auto ko_s = [&](int s) { return smem + Lay::ko_off + s * Lay::ko_bytes; };
   const int off = p.NK - p.NQ;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int us = 0, ks = 0;
-      uint32_t uph = 0, qph = 0, kph = 0;
-      uint32_t armed_q = 0, armed1[KST] = {}, armed2[KST] = {};
+      int us = 0, kst = 0, kso = 0;
+      uint32_t uph = 0, qph = 0, kpht = 0, kpho = 0;
+      uint32_t armed_q = 0, armedT[NT] = {}, armedO[NO] = {};
       int next = blockIdx.x;
       bool ok = true;
       for (;;) {
@@ -277,36 +287,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_3d(q2_s + b * (RQ * 128), &p.tmQ2, qfull, b * 64, w.q0, w.bh);
         armed_q = qph + 1;
         qph ^= 1;
-        // The other side's half of a stage is freed first (after S), this side's
-        // half only after the step's contractions: load them in that order.
-        auto load_k1 = [&](int k0) -> bool {
-          if (!mbar_wait(&kempty1[ks], kph ^ 1, ctl)) return false;
-          mbar_arrive_expect_tx(&kfull1[ks], Lay::k1_bytes);
-#pragma unroll
-          for (int b = 0; b < D1 / 64; ++b)
-            tma_load_3d(k1_s(ks) + b * (CK * 128), &p.tmK1, &kfull1[ks], b * 64, k0, w.bh);
-          armed1[ks] = kph + 1;
-          return true;
-        };
-        auto load_k2 = [&](int k0) -> bool {
-          if (!mbar_wait(&kempty2[ks], kph ^ 1, ctl)) return false;
-          mbar_arrive_expect_tx(&kfull2[ks], Lay::k2_bytes);
-#pragma unroll
-          for (int b = 0; b < D2 / 64; ++b)
-            tma_load_3d(k2_s(ks) + b * (CK * 128), &p.tmK2, &kfull2[ks], b * 64, k0, w.bh);
-          armed2[ks] = kph + 1;
-          return true;
-        };
         for (int t = 0; t < w.nsteps; ++t) {
           const int k0 = w.step(t) * CK;
-          if (SIDE == 1) {
-            if (!(ok = load_k2(k0)) || !(ok = load_k1(k0))) break;
-          } else {
-            if (!(ok = load_k1(k0)) || !(ok = load_k2(k0))) break;
+          // This side's keys first: their deeper ring was freed steps ago, so the
+          // load is issued before the producer blocks on the other side's
+          // single-stage ring, which S of the previous step frees.
+          if (!(ok = mbar_wait(&kemptyT[kst], kpht ^ 1, ctl))) break;
+          mbar_arrive_expect_tx(&kfullT[kst], Lay::kt_bytes);
+#pragma unroll
+          for (int b = 0; b < DT / 64; ++b)
+            tma_load_3d(kt_s(kst) + b * (CK * 128), tmKT, &kfullT[kst], b * 64, k0, w.bh);
+          armedT[kst] = kpht + 1;
+          if (++kst == NT) {
+            kst = 0;
+            kpht ^= 1;
           }
-          if (++ks == KST) {
-            ks = 0;
-            kph ^= 1;
+          if (!(ok = mbar_wait(&kemptyO[kso], kpho ^ 1, ctl))) break;
+          mbar_arrive_expect_tx(&kfullO[kso], Lay::ko_bytes);
+#pragma unroll
+          for (int b = 0; b < DO / 64; ++b)
+            tma_load_3d(ko_s(kso) + b * (CK * 128), tmKO, &kfullO[kso], b * 64, k0, w.bh);
+          armedO[kso] = kpho + 1;
+          if (++kso == NO) {
+            kso = 0;
+            kpho ^= 1;
           }
         }
         if (!ok) break;
@@ -316,10 +320,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         volatile int zero = 0;
         WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
         if (armed_q) mbar_wait(qfull, armed_q - 1, dctl);
-        for (int s = 0; s < KST; ++s) {
-          if (armed1[s]) mbar_wait(&kfull1[s], armed1[s] - 1, dctl);
-          if (armed2[s]) mbar_wait(&kfull2[s], armed2[s] - 1, dctl);
-        }
+        for (int s = 0; s < NT; ++s)
+          if (armedT[s]) mbar_wait(&kfullT[s], armedT[s] - 1, dctl);
+        for (int s = 0; s < NO; ++s)
+          if (armedO[s]) mbar_wait(&kfullO[s], armedO[s] - 1, dctl);
       }
     }
   } else if (warp == 1) {
@@ -334,8 +338,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint64_t qtm = sdesc_sw128(SIDE == 1 ? q1a : q2a, RQ * 128, 1024);
       const uint64_t dsk = sdesc_sw128(dsa, 16, 1024);
       const uint64_t dsm = sdesc_sw128(dsa, RQ * 128, 1024);
-      int us = 0, ks_s = 0, ks_r = 0;
-      uint32_t uph = 0, qph = 0, kph_s = 0, sph = 0, dsph = 0, dkph = 0, dqph = 0;
+      int us = 0, kst_s = 0, kso_s = 0, kst_r = 0;
+      uint32_t uph = 0, qph = 0, kpht_s = 0, kpho_s = 0, sph = 0, dsph = 0, dkph = 0, dqph = 0;
       bool ok = true;
       for (;;) {
         if (!(ok = mbar_wait(&ufull[us], uph, ctl))) break;
@@ -350,12 +354,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!(ok = mbar_wait(qfull, qph, ctl))) break;
         qph ^= 1;
         auto issue_s = [&]() -> bool {
-          if (!mbar_wait(&kfull1[ks_s], kph_s, ctl)) return false;
-          if (!mbar_wait(&kfull2[ks_s], kph_s, ctl)) return false;
+          if (!mbar_wait(&kfullO[kso_s], kpho_s, ctl)) return false;
+          if (!mbar_wait(&kfullT[kst_s], kpht_s, ctl)) return false;
           if (!mbar_wait(sempty, sph ^ 1, ctl)) return false;
           tc_fence_after();
-          const uint64_t k1d = sdesc_sw128(smem_u32(k1_s(ks_s)), 16, 1024);
-          const uint64_t k2d = sdesc_sw128(smem_u32(k2_s(ks_s)), 16, 1024);
+          const uint64_t ktd = sdesc_sw128(smem_u32(kt_s(kst_s)), 16, 1024);
+          const uint64_t kod = sdesc_sw128(smem_u32(ko_s(kso_s)), 16, 1024);
+          const uint64_t k1d = SIDE == 1 ? ktd : kod;
+          const uint64_t k2d = SIDE == 1 ? kod : ktd;
 #pragma unroll
           for (int kk = 0; kk < D1 / 16; ++kk) {
             const uint32_t o = (kk >> 2) * (RQ * 128) + (kk & 3) * 32;
@@ -369,11 +375,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                          kk > 0);
           }
           umma_commit(sfull);
-          umma_commit(&kemptyO[ks_s]);  // the other side's keys are not needed after S
+          umma_commit(&kemptyO[kso_s]);  // the other side's keys are not needed after S
           sph ^= 1;
-          if (++ks_s == KST) {
-            ks_s = 0;
-            kph_s ^= 1;
+          if (++kso_s == NO) {
+            kso_s = 0;
+            kpho_s ^= 1;
+          }
+          if (++kst_s == NT) {
+            kst_s = 0;
+            kpht_s ^= 1;
           }
           return true;
         };
@@ -389,8 +399,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tc_fence_after();
           // dQ_t += (s_t dS_t) K_t: A = dS K-major (two 64-key chunks 16 KB apart),
           // B = K_t read MN-major (64-feature chunks 16 KB apart), 8 K16 steps.
-          const uint64_t ktm =
-              sdesc_sw128(smem_u32(SIDE == 1 ? k1_s(ks_r) : k2_s(ks_r)), CK * 128, 1024);
+          const uint64_t ktm = sdesc_sw128(smem_u32(kt_s(kst_r)), CK * 128, 1024);
           const uint32_t acc0 = t > 0;
           if (p.want_dq) {
 #pragma unroll
@@ -409,8 +418,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               umma_bf16_ss(tmem_base + kColDK, sdesc_advance(qtm, kk * 2048),
                            sdesc_advance(dsm, kk * 2048), idK, kk > 0);
           }
-          umma_commit(&kemptyT[ks_r]);  // step done: keys, dS tile, dK_t^T
-          if (++ks_r == KST) ks_r = 0;
+          umma_commit(&kemptyT[kst_r]);  // step done: keys, dS tile, dK_t^T
+          if (++kst_r == NT) kst_r = 0;
         }
         if (!ok) break;
         umma_commit(dqfull);
@@ -493,7 +502,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         pks = cks;
         pkph = ckph;
-        if (++cks == KST) {
+        if (++cks == NT) {
           cks = 0;
           ckph ^= 1;
         }
@@ -529,7 +538,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int t = 0; t < w.nsteps; ++t) {
         const int k0 = w.step(t) * CK;
         if (!(ok = mbar_wait(&kemptyT[cks], ckph, ctl))) break;
-        if (++cks == KST) {
+        if (++cks == NT) {
           cks = 0;
           ckph ^= 1;
         }
@@ -620,7 +629,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 template <int D1, int D2, int SIDE>
 cudaError_t launch_t(const BwdSideParams& p, int grid, cudaStream_t stream) {
-  constexpr int smem = SideLayout<D1, D2>::alloc;
+  constexpr int smem = SideLayout<D1, D2, SIDE>::alloc;
   auto kern = streamkl_bwd_side_kernel<D1, D2, SIDE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
