@@ -1,10 +1,12 @@
 """Build libstreamkl.so in-tree with nvcc for sm_100a (cross-compiles without a GPU)."""
 from __future__ import annotations
 
+import concurrent.futures
 import os
 import shutil
 import subprocess
 import sys
+import tempfile
 from pathlib import Path
 
 PKG = Path(__file__).resolve().parent
@@ -42,12 +44,23 @@ def _stale(out: Path) -> bool:
 
 
 def build(force: bool = False, extra: list[str] | None = None, out: Path = LIB) -> Path:
+    """Compile every source to an object in parallel, then link the shared library."""
     if not force and not extra and not _stale(out):
         return out
     tmp = out.with_name(out.name + f".tmp{os.getpid()}")
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), f"-I{INCLUDE}", f"-I{CSRC}",
-           *map(str, sources()), "-o", str(tmp)]
-    subprocess.run(cmd, check=True)
+    flags = [*NVCC_FLAGS, *(extra or []), f"-I{INCLUDE}", f"-I{CSRC}"]
+    compile_flags = [f for f in flags if f not in ("-shared", "-cudart", "shared")]
+    with tempfile.TemporaryDirectory(prefix="streamkl_build_") as objdir:
+        objs = [Path(objdir) / (src.stem + ".o") for src in sources()]
+        jobs = [[nvcc(), *compile_flags, "-c", str(src), "-o", str(obj)]
+                for src, obj in zip(sources(), objs)]
+        workers = max(1, min(len(jobs), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(workers) as pool:
+            for res in pool.map(lambda c: subprocess.run(c, capture_output=True, text=True), jobs):
+                sys.stderr.write(res.stdout + res.stderr)
+                if res.returncode != 0:
+                    raise subprocess.CalledProcessError(res.returncode, res.args)
+        subprocess.run([nvcc(), *flags, *map(str, objs), "-o", str(tmp)], check=True)
     os.replace(tmp, out)
     return out
 

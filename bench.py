@@ -128,6 +128,7 @@ PROFILED_SOURCES = {
     "bwd_fused_key_tiles_kernel": "bwd_sm100.cu",
     "bwd_fused_query_tiles_kernel": "bwd_qt_sm100.cu",
     "bwd_split_kernel": "bwd_split_sm100.cu",
+    "bwd_fused_sides_kernel": "bwd_side_sm100.cu",
 }
 
 
