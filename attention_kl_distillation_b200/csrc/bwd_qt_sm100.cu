@@ -23,11 +23,13 @@
 //   work unit   (bh, 128-query tile); inner loop over the 64-key steps it sees
 //   warp 0      TMA producer: Q1/Q2 tile per unit, K1/K2 tiles per step into
 //               a ring; fetches the next unit index and publishes it
-//   warp 1      TMEM owner and UMMA issuer, per step:
-//                 S1 = Q1 K1^T, S2 = Q2 K2^T                (M=128 queries, N=64)
+//   warp 1      TMEM owner; issues the contractions of each step:
 //                 dQ_t += dS_t K_t                          (M=128 queries, N=d_t)
 //                 dK_t^T = Q_t^T dS_t                       (M=d_t, N=64 keys)
-//               S of step t+1 is issued before the contractions of step t.
+//   warp 14     issues S1 = Q1 K1^T, S2 = Q2 K2^T of each step (M=128 queries,
+//               N=64), as soon as the key tile is in and the dS warps have read
+//               the previous S out; the two issuing threads keep the tensor
+//               pipe fed while the other waits on a barrier.
 //   warps 2..9  two dS warpgroups, each for 32 of the 64 keys of a step:
 //               thread r owns query row r (TMEM lane r), loads its S1 and S2
 //               segments, regenerates P1, P2 (exp2 on the MUFU pipe, packed
@@ -62,7 +64,8 @@ constexpr int CK = kBwdQtKeys;  // keys per step
 constexpr int NDS = 2;          // dS warpgroups per CTA
 constexpr int KPW = CK / NDS;   // keys of a step per dS warpgroup
 constexpr int DK_WARP0 = 2 + 4 * NDS;
-constexpr int NTHREADS = (DK_WARP0 + 4) * 32;
+constexpr int S_WARP = DK_WARP0 + 4;  // issues the S products
+constexpr int NTHREADS = (S_WARP + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS1 = 0, kColS2 = 64, kColDQ1 = 128, kColDK1 = 384, kColDK2 = 448;
@@ -281,9 +284,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(dqempty, 4);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ufull[s], 1);
-      mbar_init(&uempty[s], 1 + 4 * NDS + 4);  // MMA thread + dS warps + dK warps
+      mbar_init(&uempty[s], 2 + 4 * NDS + 4);  // both UMMA issuers + dS warps + dK warps
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);
     fence_mbar_init();
     tma_prefetch_desc(&p.tmQ1);
     tma_prefetch_desc(&p.tmK1);
@@ -366,9 +369,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (armed_k[s]) mbar_wait(&kfull[s], armed_k[s] - 1, dctl);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
+  } else if (warp == 1 || warp == S_WARP) {
+    // ------------------------------------------------------------ UMMA issuers
+    // Two threads feed the tensor pipe: the S products come from warp S_WARP,
+    // the contractions from warp 1.  The queue in front of the pipe holds about
+    // one product, so a single issuing thread leaves the pipe idle whenever it
+    // checks a barrier or waits; with two, one stream's waits are filled by the
+    // other's products.  A commit tracks the issuing thread's own products,
+    // which is what each barrier below means: sfull the S of a step, kempty the
+    // contractions of a step (whose dS implies that step's S was done).
     if (lane == 0) {
+      const bool s_role = warp == S_WARP;
       constexpr uint32_t idS = idesc_bf16(RQ, CK);           // S: M=128 queries, N=64 keys
       constexpr uint32_t idQ1 = idesc_bf16(RQ, D1, 0, 1);    // dQ1: B = K1 MN-major
       constexpr uint32_t idQ2 = idesc_bf16(RQ, D2, 0, 1);
@@ -394,39 +405,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         if (u < 0) break;
         const UnitQ w = decode_unit(p, u);
-        if (!(ok = mbar_wait(qfull, qph, ctl))) break;
-        qph ^= 1;
-        auto issue_s = [&]() -> bool {
-          if (!mbar_wait(&kfull[ks_s], kph_s, ctl)) return false;
-          if (!mbar_wait(&sempty[sb], ((sph >> sb) & 1u) ^ 1u, ctl)) return false;
-          tc_fence_after();
-          const uint32_t scol = tmem_base + (sb == 0 ? 0u : kColSB1);
-          const uint64_t k1d = sdesc_sw128(smem_u32(k1_s(ks_s)), 16, 1024);
-          const uint64_t k2d = sdesc_sw128(smem_u32(k2_s(ks_s)), 16, 1024);
+        if (s_role) {
+          if (!(ok = mbar_wait(qfull, qph, ctl))) break;
+          qph ^= 1;
+          for (int t = 0; t < w.nsteps; ++t) {
+            if (!(ok = mbar_wait(&kfull[ks_s], kph_s, ctl))) break;
+            if (!(ok = mbar_wait(&sempty[sb], ((sph >> sb) & 1u) ^ 1u, ctl))) break;
+            tc_fence_after();
+            const uint32_t scol = tmem_base + (sb == 0 ? 0u : kColSB1);
+            const uint64_t k1d = sdesc_sw128(smem_u32(k1_s(ks_s)), 16, 1024);
+            const uint64_t k2d = sdesc_sw128(smem_u32(k2_s(ks_s)), 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D1 / 16; ++kk) {
-            const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(scol + kColS1, sdesc_advance(q1d, (kk >> 2) * (RQ * 128) + o),
-                         sdesc_advance(k1d, (kk >> 2) * (CK * 128) + o), idS, kk > 0);
-          }
+            for (int kk = 0; kk < D1 / 16; ++kk) {
+              const uint32_t o = (kk & 3) * 32;
+              umma_bf16_ss(scol + kColS1, sdesc_advance(q1d, (kk >> 2) * (RQ * 128) + o),
+                           sdesc_advance(k1d, (kk >> 2) * (CK * 128) + o), idS, kk > 0);
+            }
 #pragma unroll
-          for (int kk = 0; kk < D2 / 16; ++kk) {
-            const uint32_t o = (kk & 3) * 32;
-            umma_bf16_ss(scol + kColS2, sdesc_advance(q2d, (kk >> 2) * (RQ * 128) + o),
-                         sdesc_advance(k2d, (kk >> 2) * (CK * 128) + o), idS, kk > 0);
+            for (int kk = 0; kk < D2 / 16; ++kk) {
+              const uint32_t o = (kk & 3) * 32;
+              umma_bf16_ss(scol + kColS2, sdesc_advance(q2d, (kk >> 2) * (RQ * 128) + o),
+                           sdesc_advance(k2d, (kk >> 2) * (CK * 128) + o), idS, kk > 0);
+            }
+            umma_commit(&sfull[sb]);
+            sph ^= 1u << sb;
+            if (NSB == 2) sb ^= 1;
+            if (++ks_s == KST) {
+              ks_s = 0;
+              kph_s ^= 1;
+            }
           }
-          umma_commit(&sfull[sb]);
-          sph ^= 1u << sb;
-          if (NSB == 2) sb ^= 1;
-          if (++ks_s == KST) {
-            ks_s = 0;
-            kph_s ^= 1;
-          }
-          return true;
-        };
-        if (!(ok = issue_s())) break;
-        for (int t = 0; t < w.nsteps && ok; ++t) {
-          if (t + 1 < w.nsteps && !(ok = issue_s())) break;
+          if (!ok) break;
+          continue;
+        }
+        for (int t = 0; t < w.nsteps; ++t) {
           if (!(ok = mbar_wait(&dsfull[db], dsph[db], ctl))) break;
           dsph[db] ^= 1;
           if (t == 0) {  // the previous unit's dQ has been read out of TMEM
@@ -435,9 +447,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           tc_fence_after();
           // Descriptors of this step's operands are built once; each UMMA below
-          // adds a constant offset.  The single issuing thread needs about as long
-          // to issue an M128 N64 product as the tensor pipe takes to run an N128
-          // one, so little else may sit between the issues.
+          // adds a constant offset.
           const uint32_t ds1a = smem_u32(ds1_s(db)), ds2a = smem_u32(ds2_s(db));
           const uint64_t d1k = sdesc_sw128(ds1a, 16, 1024), d2k = sdesc_sw128(ds2a, 16, 1024);
           const uint64_t d1m = sdesc_sw128(ds1a, CK * 128, 1024), d2m = sdesc_sw128(ds2a, CK * 128, 1024);
@@ -490,6 +500,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         umma_commit(dqfull);
         umma_commit(qempty);
       }
+      // each issuer's products are complete before TMEM is released (drain counts both)
       umma_commit(drain);
       volatile int zero = 0;
       WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
