@@ -200,9 +200,9 @@ int bwd_algo_setting() {
 // AUTO: the page keeps the fused kernel while its atomic reductions stay cheap
 // and switches to separate kernels when they contend.  On B200 the fused
 // kernels measured faster at every size tested, in or beyond L2: B1 H32 N16384
-// d128 causal (537 MB fp32 accumulator) fused query tiles 8.17 ms, fused key
-// tiles 9.43, split 10.37; B1 H80 N65536 d128 causal (5 GiB accumulator)
-// 357, 365 and 400 ms (bench.py --compare-bwd).  So AUTO is FUSED at every
+// d128 causal (537 MB fp32 accumulator) fused query tiles 8.2-8.6 ms, fused
+// key tiles 9.4-9.7, split 10.4-10.7; B1 H80 N65536 d128 causal (5 GiB
+// accumulator) 357, 365 and 400 ms (bench.py --compare-bwd).  So AUTO is FUSED at every
 // size; SPLIT stays available explicitly.
 
 // SMs of the current device for scheduling decisions; 148 (B200) when no
@@ -559,8 +559,9 @@ streamkl_status streamkl_bwd(const streamkl_problem* prob, const float* dL, cons
   const int sel = ((dQ1 || dK1) ? 1 : 0) | ((dQ2 || dK2) ? 2 : 0);
   streamkl_bwd_algorithm algo = resolve_bwd_algo(*prob);
   // AUTO and FUSED run one side alone with 128-key steps when only one side is
-  // asked for (B1 H32 N16384 d128 causal, student side: 5.77 against 6.14 ms
-  // for the query-tile kernel's one-sided instance); an explicit setting is kept.
+  // asked for (B1 H32 N16384 d128 causal: student side 4.89 against 6.14 ms for
+  // the query-tile kernel's one-sided instance, teacher side 4.90 against 6.30);
+  // an explicit setting is kept.
   const int setting = bwd_algo_setting();
   if (algo == STREAMKL_BWD_FUSED_QUERY_TILES && sel != 3 &&
       (setting == STREAMKL_BWD_AUTO || setting == STREAMKL_BWD_FUSED))
