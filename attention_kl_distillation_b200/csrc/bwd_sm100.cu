@@ -14,12 +14,13 @@
 //   warp 0      TMA producer: K1/K2 tile per unit; Q1/Q2 tile + per-row record
 //               (LSE1, LSE2, L, s*dL) per step into a 2-stage ring; also
 //               fetches the next unit index and publishes it to the other roles
-//   warp 1      TMEM owner and UMMA issuer, per step:
-//                 S1^T = K1 Q1^T, S2^T = K2 Q2^T           (M=128 keys, N=64)
+//   warp 1      TMEM owner; issues the contractions of each step:
 //                 dK_t += dS_t^T Q_t                        (M=128 keys, N=d_t)
 //                 dQ_t^T = K_t^T dS_t^T                     (M=d_t, N=64 queries)
-//               S for step t+1 is issued before the contractions of step t so
-//               that the tensor pipe works while dS is being formed.
+//   warp 14     issues S1^T = K1 Q1^T, S2^T = K2 Q2^T of each step (M=128 keys,
+//               N=64) as soon as the query tile is in and the dS warps have read
+//               the previous S out, so the tensor pipe works on S of step t+1
+//               while dS of step t is formed and while warp 1 waits.
 //   warps 2..9  two dS warpgroups, each for 32 of the 64 queries of a step:
 //               thread j owns key j (TMEM lane j), loads its S1^T and S2^T
 //               row segments, regenerates P1, P2 with exp2 on the MUFU pipe
@@ -57,7 +58,8 @@ constexpr int BQ = kBwdBQ;  // queries per step
 constexpr int NDS = 2;          // dS warpgroups per CTA
 constexpr int QPW = BQ / NDS;   // queries of a step per dS warpgroup
 constexpr int DQ_WARP0 = 2 + 4 * NDS;
-constexpr int NTHREADS = (DQ_WARP0 + 4) * 32;
+constexpr int S_WARP = DQ_WARP0 + 4;  // issues the S^T products
+constexpr int NTHREADS = (S_WARP + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kColS1 = 0, kColS2 = 64, kColDK1 = 128, kColDQ1 = 384, kColDQ2 = 448;
 
@@ -285,9 +287,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
     mbar_init(dkempty, 4);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ufull[s], 1);
-      mbar_init(&uempty[s], 1 + 4 * NDS + 4);  // MMA thread + dS warps + dQ warps
+      mbar_init(&uempty[s], 2 + 4 * NDS + 4);  // both UMMA issuers + dS warps + dQ warps
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);
     fence_mbar_init();
     tma_prefetch_desc(&p.tmQ1);
     tma_prefetch_desc(&p.tmK1);
@@ -380,9 +382,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           if (armed_q[s]) mbar_wait(&qfull[s], armed_q[s] - 1, dctl);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
+  } else if (warp == 1 || warp == S_WARP) {
+    // ------------------------------------------------------------ UMMA issuers
+    // The S^T products come from warp S_WARP, the contractions from warp 1 (the
+    // queue in front of the tensor pipe holds about one product, so one
+    // stream's barrier waits are filled by the other's products).  Each commit
+    // tracks its own thread's products; the contractions of a step imply its
+    // S^T (their dS was formed from it), so the stage and unit releases below
+    // stay with warp 1.
     if (lane == 0) {
+      const bool s_role = warp == S_WARP;
       constexpr uint32_t idS = idesc_bf16(BK, BQ);                // S^T: M=128 keys, N=64
       constexpr uint32_t idK1 = idesc_bf16(BK, D1, 0, 1);         // dK1: B = Q1 MN-major
       constexpr uint32_t idK2 = idesc_bf16(BK, D2, 0, 1);
@@ -407,8 +416,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         }
         if (u < 0) break;
         const UnitB w = decode_unit(p, u);
-        if (!(ok = mbar_wait(kfull, kph, ctl))) break;
-        kph ^= 1;
+        if (s_role) {
+          if (!(ok = mbar_wait(kfull, kph, ctl))) break;
+          kph ^= 1;
+        }
         auto issue_s = [&]() -> bool {
           if (!mbar_wait(&qfull[qs_s], qph_s, ctl)) return false;
           if (!mbar_wait(sempty, sph ^ 1, ctl)) return false;
@@ -435,9 +446,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
           }
           return true;
         };
-        if (!(ok = issue_s())) break;
+        if (s_role) {
+          for (int t = 0; t < w.nsteps && ok; ++t) ok = issue_s();
+          if (!ok) break;
+          continue;
+        }
         for (int t = 0; t < w.nsteps && ok; ++t) {
-          if (t + 1 < w.nsteps && !(ok = issue_s())) break;
           if (!(ok = mbar_wait(&dsfull[db], dsph[db], ctl))) break;
           dsph[db] ^= 1;
           if (t == 0) {
@@ -497,6 +511,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) streamkl_bwd_kernel(const __grid_
         umma_commit(dkfull);
         umma_commit(kempty);
       }
+      // each issuer's products are complete before TMEM is released (drain counts both)
       umma_commit(drain);
       volatile int zero = 0;
       WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
