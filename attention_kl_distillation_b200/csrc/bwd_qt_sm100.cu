@@ -500,11 +500,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         umma_commit(dqfull);
         umma_commit(qempty);
       }
-      // each issuer's products are complete before TMEM is released (drain counts both)
+      // Every product of both issuers is complete before TMEM is released: drain
+      // counts a commit from each, and warp 1, which releases TMEM after the
+      // final barrier, waits for it.  The S issuer, which may finish a unit
+      // ahead, does not wait (its wait would span warp 1's whole last unit).
       umma_commit(drain);
-      volatile int zero = 0;
-      WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
-      mbar_wait(drain, 0, dctl);
+      if (!s_role) {
+        volatile int zero = 0;
+        WaitCtl dctl{&zero, p.status, p.wait_limit_ns};
+        mbar_wait(drain, 0, dctl);
+      }
     }
   } else if (warp < DK_WARP0) {
     // ------------------------------------------------------------ dS warpgroups
